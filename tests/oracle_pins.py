@@ -1,0 +1,207 @@
+"""Pins for the fp64 oracle: checks against facts fixed outside the oracle itself.
+
+Each check takes the oracle module as an argument, so that the same checks can be
+run against deliberately broken copies of the oracle (see test_oracle_mutations.py)
+to show that a plausible mistake is caught.
+
+Sources of truth used here:
+  * hand-worked examples of Eqs. (1), (2), (4), (7)-(12) in tests/golden/
+    ("MISA: Mixture of Indexer Sparse Attention", Introduction and Methodology);
+  * closed forms (the mean of an arithmetic progression of keys);
+  * library routines for selection (heapq.nlargest) and a brute-force rank count;
+  * structural invariants of the equations: h = H^I turns Eq. (9) into Eq. (1);
+    k' >= P turns MISA-dagger into the dense TopK; scaling or sign-flipping w
+    leaves the routed head set unchanged (|A| in Eq. 7).
+"""
+
+from __future__ import annotations
+
+import heapq
+
+import numpy as np
+
+from tests.golden import fixtures
+
+
+def _q(fx, H, d):
+    return fx["q"].reshape(H, d)
+
+
+# ----------------------------------------------------------------- hand-worked examples
+def check_dense_hand(orc):
+    fx = fixtures.load("eq1_dense_hand.txt")
+    H, d, L = int(fx["H"][0]), int(fx["d"][0]), int(fx["L"][0])
+    q, w, k = _q(fx, H, d), fx["w"], fx["k"].reshape(L, d)
+    I = orc.dense_scores(q, w, k, L)
+    assert np.array_equal(I, fx["I"]), (I, fx["I"])
+    idx, vals = orc.topk(I, 3)
+    assert list(idx) == [int(x) for x in fx["top3"]], idx
+    assert np.array_equal(orc.token_scores(q, w, k, L, [0]), fx["routed_h0"])
+    assert np.array_equal(orc.token_scores(q, w, k, L, [1]), fx["routed_h1"])
+
+
+def check_router_hand(orc):
+    fx = fixtures.load("eq7_router_hand.txt")
+    H, d, B, L = int(fx["H"][0]), int(fx["d"][0]), int(fx["B"][0]), int(fx["L"][0])
+    P = int(fx["pos"][0]) + 1
+    q, w, k = _q(fx, H, d), fx["w"], fx["k"].reshape(L, d)
+    kp = orc.pool_keys(k[:P], B)
+    assert np.array_equal(kp, fx["kpool"].reshape(-1, d)), kp
+    E = orc.router_energy(q, w, k, P, B)
+    assert np.allclose(E, fx["E"], rtol=0, atol=1e-15), E
+    assert list(orc.select_heads(E, H)) == [int(x) for x in fx["heads"]]
+    r = orc.misa_row(q, w, k, P, B, 2, 5)
+    assert list(r["heads"]) == [1, 0]
+    assert np.array_equal(r["scores"], fx["routed_h2"]), r["scores"]
+    assert list(r["idx"]) == [int(x) for x in fx["routed_h2_top5"]], r["idx"]
+    assert np.array_equal(orc.dense_scores(q, w, k, P), fx["dense"])
+    r1 = orc.misa_row(q, w, k, P, B, 1, 1)
+    assert list(r1["heads"]) == [int(x) for x in fx["h1_heads"]]
+    assert list(r1["idx"]) == [int(x) for x in fx["h1_misa_top1"]], r1["idx"]
+    omega, _ = orc.topk(r1["scores"], 3)
+    assert list(omega) == [int(x) for x in fx["h1_omega_k3"]], omega
+    dg = orc.misa_dagger_row(q, w, k, P, omega, 1)
+    assert list(dg["idx"]) == [int(x) for x in fx["h1_dagger_top1"]], dg["idx"]
+    assert list(orc.dsa_row(q, w, k, P, 1)["idx"]) == [int(x) for x in fx["h1_dagger_top1"]]
+
+
+# ----------------------------------------------------------------- closed forms
+def check_pool_closed_form(orc):
+    # keys k_s = s (every dim): block b's mean is the midpoint of its first and last index
+    for L, B in [(10, 4), (64, 64), (65, 64), (7, 3), (1, 5), (130, 128)]:
+        k = np.repeat(np.arange(L, dtype=np.float64)[:, None], 3, axis=1)
+        kp = orc.pool_keys(k, B)
+        M = -(-L // B)
+        assert kp.shape == (M, 3)
+        for b in range(M):
+            first, last = b * B, min((b + 1) * B, L) - 1
+            assert np.all(kp[b] == (first + last) / 2.0), (L, B, b, kp[b])
+    # B = 1: pooling is the identity
+    rng = np.random.default_rng(1)
+    k = rng.standard_normal((37, 8))
+    assert np.array_equal(orc.pool_keys(k, 1), k)
+
+
+def check_router_closed_form(orc):
+    """q_j = a_j * e_j, all keys equal to the all-ones vector: every pooled key is the
+    all-ones vector, so E_j = |w_j| * ReLU(a_j) for any prefix length and block size."""
+    H, d = 6, 6
+    a = np.array([3.0, -1.0, 0.5, 2.0, 0.0, 1.5])
+    w = np.array([0.25, 4.0, -2.0, -0.5, 1.0, 1.0])
+    q = np.diag(a)
+    k = np.ones((50, d))
+    for P, B in [(1, 4), (5, 4), (8, 4), (50, 7), (50, 64)]:
+        E = orc.router_energy(q, w, k, P, B)
+        assert np.allclose(E, np.abs(w) * np.maximum(a, 0.0), rtol=1e-15, atol=0), (P, B, E)
+    E = orc.router_energy(q, w, k, 50, 7)
+    # E = [0.75, 0, 1.0, 1.0, 0, 1.5] -> descending with lower index first on ties
+    assert list(orc.select_heads(E, 6)) == [5, 2, 3, 0, 1, 4]
+
+
+def check_partial_block_router(orc):
+    """A query whose prefix ends mid-block routes on the mean of the block's valid keys
+    only.  Keys k_s = s * u with u a unit vector; the partial block {8, 9} of P = 10,
+    B = 4 pools to 8.5 * u (a full-L pooling would give 9.5 * u, an unweighted sum 17 * u)."""
+    d = 4
+    u = np.array([1.0, 0.0, 0.0, 0.0])
+    k = np.arange(12, dtype=np.float64)[:, None] * u[None, :]
+    q = np.array([[1.0, 0, 0, 0]])
+    w = np.array([1.0])
+    E = orc.router_energy(q, w, k, 10, 4)
+    # pooled keys of the prefix: 1.5, 5.5, 8.5 (times u); E = (1.5 + 5.5 + 8.5) / 3
+    assert abs(E[0] - (1.5 + 5.5 + 8.5) / 3.0) < 1e-14, E
+
+
+# ----------------------------------------------------------------- library routine / brute force
+def check_topk_against_library(orc):
+    rng = np.random.default_rng(2)
+    for n, kk in [(1, 1), (5, 3), (40, 7), (200, 64), (13, 20), (300, 300)]:
+        # quantised values so that ties are frequent
+        s = np.round(rng.standard_normal(n) * 4) / 4
+        idx, vals = orc.topk(s, kk)
+        ref = heapq.nlargest(min(kk, n), range(n), key=lambda i: (s[i], -i))
+        assert list(idx[:len(ref)]) == ref, (n, kk)
+        assert np.all(idx[len(ref):] == -1) and np.all(np.isneginf(vals[len(ref):]))
+        assert np.array_equal(vals[:len(ref)], s[ref])
+
+
+def check_topk_brute_rank(orc):
+    """Brute force: item i is selected iff fewer than k items beat it, where j beats i
+    when s_j > s_i, or s_j == s_i and j < i."""
+    rng = np.random.default_rng(3)
+    for n, kk in [(9, 4), (16, 16), (25, 1), (30, 12)]:
+        s = rng.integers(-3, 4, size=n).astype(np.float64)
+        idx, _ = orc.topk(s, kk)
+        chosen = set(int(i) for i in idx if i >= 0)
+        for i in range(n):
+            beats = sum(1 for j in range(n) if s[j] > s[i] or (s[j] == s[i] and j < i))
+            assert (beats < kk) == (i in chosen), (n, kk, i)
+
+
+# ----------------------------------------------------------------- invariants
+def _rand_problem(seed, H=8, d=16, L=97):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((H, d))
+    w = rng.standard_normal(H)
+    k = rng.standard_normal((L, d)) + 0.3 * rng.standard_normal((1, d))
+    return q, w, k
+
+
+def check_h_equals_H_is_dense(orc):
+    for seed in range(4):
+        q, w, k = _rand_problem(seed)
+        H = q.shape[0]
+        for P in (1, 17, 97):
+            r = orc.misa_row(q, w, k, P, 8, H, 10)
+            dd = orc.dsa_row(q, w, k, P, 10)
+            assert np.array_equal(r["scores"], dd["scores"])
+            assert np.array_equal(r["idx"], dd["idx"])
+
+
+def check_dagger_limits(orc):
+    for seed in range(4):
+        q, w, k = _rand_problem(seed + 10)
+        for P in (5, 60, 97):
+            r = orc.misa_row(q, w, k, P, 8, 3, 10)
+            # k' >= P: the candidate set is the whole prefix -> exactly the dense TopK
+            cand, _ = orc.topk(r["scores"], max(P, 12))
+            dg = orc.misa_dagger_row(q, w, k, P, cand, 10)
+            assert np.array_equal(dg["idx"], orc.dsa_row(q, w, k, P, 10)["idx"])
+            # k' = k: the re-rank keeps MISA's set (order may change)
+            cand, _ = orc.topk(r["scores"], 10)
+            dg = orc.misa_dagger_row(q, w, k, P, cand, 10)
+            assert set(dg["idx"].tolist()) == set(r["idx"].tolist())
+
+
+def check_router_w_invariance(orc):
+    for seed in range(4):
+        q, w, k = _rand_problem(seed + 20)
+        E = orc.router_energy(q, w, k, 90, 8)
+        heads = orc.select_heads(E, 3)
+        E2 = orc.router_energy(q, 2.5 * w, k, 90, 8)
+        assert np.allclose(E2, 2.5 * E, rtol=1e-13, atol=0)
+        assert np.array_equal(orc.select_heads(E2, 3), heads)
+        E3 = orc.router_energy(q, -w, k, 90, 8)
+        assert np.array_equal(E3, E)
+        perm = np.random.default_rng(seed).permutation(q.shape[0])
+        E4 = orc.router_energy(q[perm], w[perm], k, 90, 8)
+        assert np.allclose(E4, E[perm], rtol=1e-13, atol=0)
+
+
+def check_causal_prefix(orc):
+    """Keys after the query's position never influence its scores or its routing."""
+    q, w, k = _rand_problem(30, L=80)
+    k2 = k.copy()
+    k2[50:] = 1e3
+    r1 = orc.misa_row(q, w, k, 50, 8, 3, 10)
+    r2 = orc.misa_row(q, w, k2, 50, 8, 3, 10)
+    assert np.array_equal(r1["E"], r2["E"]) and np.array_equal(r1["idx"], r2["idx"])
+    assert r1["scores"].shape == (50,)
+
+
+ALL_CHECKS = [
+    check_dense_hand, check_router_hand, check_pool_closed_form, check_router_closed_form,
+    check_partial_block_router, check_topk_against_library, check_topk_brute_rank,
+    check_h_equals_H_is_dense, check_dagger_limits, check_router_w_invariance,
+    check_causal_prefix,
+]

@@ -1,0 +1,367 @@
+"""Benchmark of the MISA indexer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the MISA path over one batch of synthetic input that is
+already resident in HBM: block pooling (Eq. 4), head routing (Eqs. 7-8), routed
+scoring and top-k (Eqs. 9-10).  The dense DSA indexer (Eqs. 1-2) and MISA-dagger
+(coarse top-k' + all-head re-rank, Eqs. 11-12) run the same number of steps on the
+same inputs, timed separately, and are reported beside it.  Rank 0 prints one JSON
+line.  Throughput unit: query x prefix-token pairs scored per second.
+
+Inputs are larger than L2 (126 MB) and two copies are used alternately, so no step
+reads keys another step left in L2.
+
+`--impl reference` times the fp64 CPU oracle (the parity reference) on a bounded
+sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "indexer query×prefix-tokens/s at 32K–128K (MISA h=8 vs dense); % of roofline"
+UNIT = "query×prefix-tokens/s"
+DEFAULT_WORKLOAD = "dsv32_decode_32k"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def _dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_bytes_score(wl) -> float:
+    """Bytes the routed score + top-k call must move: every key of every query's prefix
+    (256 B per token per query row -- decode rows do not share keys), the routed query
+    vectors, and the selected indices/values."""
+    P = wl.positions().astype(np.int64) + 1
+    if wl.T == 1:
+        keys = float(P.sum()) * wl.d * 2
+    else:
+        keys = float(wl.nseq) * wl.L * wl.d * 2   # one sequence's keys shared by its queries
+    return keys + wl.rows * (wl.h * wl.d * 2 + wl.h * 4 + wl.H * 4) + wl.rows * wl.topk * 8
+
+
+def run_reference(args, wl):
+    """fp64 CPU oracle on a bounded sample: each step = one query row of the workload."""
+    rank, world, _ = _dist_env()
+    if rank != 0:
+        return 0
+    import oracle.misa_oracle as orc
+    from threadpoolctl import threadpool_info
+    x = make_inputs(wl, seed=0)
+    rows = list(range(wl.rows))
+    T = wl.T
+
+    def one(row):
+        n, t = divmod(row, T)
+        k = orc.bf16_bits_to_f64(x.k_bits[n])
+        q_t = orc.bf16_bits_to_f64(x.q_bits[n, t])
+        P = int(x.pos[n, t]) + 1
+        orc.misa_row(q_t, x.w[n, t].astype(np.float64), k, P, wl.B, wl.h, wl.topk)
+        return P
+
+    for i in range(args.warmup):
+        one(rows[i % len(rows)])
+    t0 = time.perf_counter()
+    units = 0
+    for i in range(args.steps):
+        units += one(rows[(args.warmup + i) % len(rows)])
+    dt = time.perf_counter() - t0
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    val = units / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "nseq": wl.nseq, "T": wl.T, "L": wl.L, "H": wl.H,
+                   "h": wl.h, "B": wl.B, "topk": wl.topk, "path": "MISA (pool+route+score+top-k)"},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{args.steps} query rows of {wl.name} (one row per step), "
+                                   "fp64 numpy oracle"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def cpu_baseline(wl, budget_s: float = 12.0):
+    """Time the oracle's MISA path on the host cores over as many rows as fit the budget."""
+    import oracle.misa_oracle as orc
+    from threadpoolctl import threadpool_info
+    x = make_inputs(wl.replace(nseq=min(wl.nseq, 8)) if wl.T == 1 else wl, seed=0)
+    units, rows_done = 0, 0
+    t0 = time.perf_counter()
+    for row in range(x.wl.rows):
+        n, t = divmod(row, x.wl.T)
+        k = orc.bf16_bits_to_f64(x.k_bits[n])
+        q_t = orc.bf16_bits_to_f64(x.q_bits[n, t])
+        P = int(x.pos[n, t]) + 1
+        orc.misa_row(q_t, x.w[n, t].astype(np.float64), k, P, wl.B, wl.h, wl.topk)
+        units += P
+        rows_done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    return {"value": units / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows_done} query rows of {wl.name} ({units} query x prefix-token pairs), "
+                      f"full MISA path in fp64 numpy, {dt:.1f} s"}
+
+
+def run_cuda(args, wl):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=dev)
+    import long_context_block_b200 as M
+    peaks = _peaks()
+
+    x = make_inputs(wl, seed=rank)
+    q_h = torch.from_numpy(x.q_bits.view(np.int16)).pin_memory()
+    k_h = torch.from_numpy(x.k_bits.view(np.int16)).pin_memory()
+    w_h = torch.from_numpy(x.w).pin_memory()
+    pos_h = torch.from_numpy(x.pos.astype(np.int32)).pin_memory()
+    sets = []
+    for _ in range(2):   # two resident copies, used alternately (each larger than L2)
+        sets.append((q_h.to(dev).view(torch.bfloat16), w_h.to(dev),
+                     k_h.to(dev).view(torch.bfloat16), pos_h.to(dev)))
+    nseq, T, H, d = wl.nseq, wl.T, wl.H, wl.d
+    M_blocks = -(-wl.L // wl.B)
+    kp = [torch.empty((nseq, M_blocks, d), dtype=torch.float32, device=dev) for _ in range(2)]
+    heads = torch.empty((nseq, T, wl.h), dtype=torch.int32, device=dev)
+    idx = torch.empty((nseq, T, wl.topk), dtype=torch.int32, device=dev)
+    vals = torch.empty((nseq, T, wl.topk), dtype=torch.float32, device=dev)
+    cand = torch.empty((nseq, T, wl.kprime), dtype=torch.int32, device=dev)
+    gidx = torch.empty_like(idx)
+    gvals = torch.empty_like(vals)
+    didx = torch.empty_like(idx)
+    dvals = torch.empty_like(vals)
+    units = wl.query_prefix_tokens()
+    stream = torch.cuda.current_stream()
+
+    ev_score = []   # (start, end) around the routed score + top-k call
+
+    def misa_step(i, record=False):
+        q, w, k, pos = sets[i % 2]
+        M.misa_pool_keys(k, wl.B, out=kp[i % 2])
+        M.misa_route_heads(q, w, k, kp[i % 2], pos, wl.B, wl.h, heads=heads)
+        if record:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        M.misa_score_topk(q, w, k, heads, pos, wl.topk, idx=idx, vals=vals)
+        if record:
+            b.record(stream)
+            ev_score.append((a, b))
+
+    def dagger_step(i):
+        q, w, k, pos = sets[i % 2]
+        M.misa_pool_keys(k, wl.B, out=kp[i % 2])
+        M.misa_route_heads(q, w, k, kp[i % 2], pos, wl.B, wl.h, heads=heads)
+        M.misa_score_topk(q, w, k, heads, pos, wl.kprime, return_vals=False, idx=cand)
+        M.misa_dagger_rerank(q, w, k, pos, cand, wl.topk, idx=gidx, vals=gvals)
+
+    def dsa_step(i):
+        q, w, k, pos = sets[i % 2]
+        M.dsa_score_topk(q, w, k, pos, wl.topk, idx=didx, vals=dvals)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(step_fn, steps, warmup, **kw):
+        for i in range(warmup):
+            step_fn(i)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            step_fn(warmup + i, **kw)
+        e1.record(stream)
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms / steps
+
+    with ClockSampler(local) as clk:
+        ms_misa = timed(misa_step, args.steps, args.warmup, record=True)
+    clocks = clk.summary()
+    M.misa_check_device_status(dev)
+    score_ms = [a.elapsed_time(b) for a, b in ev_score]
+    score_ms_avg = sum(score_ms) / len(score_ms)
+    ms_dagger = timed(dagger_step, args.steps, args.warmup)
+    ms_dsa = timed(dsa_step, args.steps, args.warmup)
+    M.misa_check_device_status(dev)
+
+    # end to end through the public API: pinned host inputs -> device -> MISA -> host indices
+    idx_h = torch.empty((nseq, T, wl.topk), dtype=torch.int32).pin_memory()
+    e2e_dev = [torch.empty_like(t) for t in sets[0]]
+
+    def e2e_step(i):
+        for dst, src in zip(e2e_dev, (q_h, w_h, k_h, pos_h)):
+            dst.view(src.dtype).copy_(src, non_blocking=True)
+        q, w, k, pos = e2e_dev
+        out_idx, _, _ = M.misa_indexer(q, w, k, pos, wl.B, wl.h, wl.topk)
+        idx_h.copy_(out_idx, non_blocking=True)
+
+    ms_e2e = timed(e2e_step, max(3, args.steps // 2), 2)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, w_h, k_h, pos_h))
+    d2h = idx_h.numel() * idx_h.element_size()
+
+    score_bytes = algorithmic_bytes_score(wl)
+    achieved = score_bytes / (score_ms_avg * 1e-3) / 1e9
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        with open(tfile) as f:
+            traffic = json.load(f).get(wl.name, {}).get("misa_score_topk")
+
+    line = {
+        "metric": METRIC, "value": units * world / (ms_misa * 1e-3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_misa,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "nseq": nseq, "T": T, "L": wl.L, "H": H, "d": d,
+                   "h": wl.h, "B": wl.B, "topk": wl.topk, "kprime": wl.kprime,
+                   "path": "MISA: pool + route + routed score + top-k",
+                   "l2": "inputs > L2 (keys %.0f MB), two resident copies used alternately"
+                         % (x.k_bits.nbytes / 1e6),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": {"kernel": "misa_score_topk (routed score + top-k)", "bound": "hbm",
+                     "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm"], "traffic": traffic,
+                     "peak_source": peaks["source"], "algorithmic_bytes": score_bytes,
+                     "avg_ms": score_ms_avg},
+        "paths": {
+            "misa": {"value": units * world / (ms_misa * 1e-3), "ms_per_step": ms_misa},
+            "dsa": {"value": units * world / (ms_dsa * 1e-3), "ms_per_step": ms_dsa},
+            "misa_dagger": {"value": units * world / (ms_dagger * 1e-3), "ms_per_step": ms_dagger},
+            "speedup_misa_vs_dsa": ms_dsa / ms_misa,
+            "speedup_dagger_vs_dsa": ms_dsa / ms_dagger,
+        },
+        "e2e": {"value": units * world / (ms_e2e * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_cuda(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,259 @@
+// C ABI of the MISA indexer library: argument validation, workspace layout and the
+// launch sequence of each entry point.  Declarations and contracts: include/misa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "misa.h"
+
+using namespace misa;
+
+namespace {
+
+using GetRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+GetRangeFn get_range_fn() {
+  static GetRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetRangeFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// A device buffer of at least `bytes` bytes, `align`-aligned, allocated on a CUDA device.
+int check_dev(const void* p, size_t bytes, size_t align) {
+  if (p == nullptr) return MISA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p) % align) return MISA_ERR_INVALID_ARG;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return MISA_ERR_INVALID_ARG;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return MISA_ERR_INVALID_ARG;
+  if (a.type == cudaMemoryTypeDevice) {
+    if (GetRangeFn fn = get_range_fn()) {
+      CUdeviceptr base = 0;
+      size_t size = 0;
+      if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(p)) == CUDA_SUCCESS) {
+        if (reinterpret_cast<uintptr_t>(p) + bytes > (uintptr_t)base + size)
+          return MISA_ERR_INVALID_ARG;
+      }
+    }
+  }
+  return MISA_OK;
+}
+int check_opt(const void* p, size_t bytes, size_t align) {
+  return p == nullptr ? MISA_OK : check_dev(p, bytes, align);
+}
+
+#define MISA_TRY(expr)            \
+  do {                            \
+    const int _s = (expr);        \
+    if (_s != MISA_OK) return _s; \
+  } while (0)
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA; }
+
+// Shape checks shared by all query-side entry points (host-only, no CUDA calls).
+int check_shape(int nseq, int T, int H, int d, int64_t L) {
+  if (nseq < 1 || T < 1 || H < 1 || d < 1 || L < 1) return MISA_ERR_INVALID_ARG;
+  if (L >= INT32_MAX || (int64_t)nseq * T >= INT32_MAX) return MISA_ERR_INVALID_ARG;
+  if (d != MISA_HEAD_DIM || H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
+  return MISA_OK;
+}
+int check_topk(int topk) {
+  if (topk < 1) return MISA_ERR_INVALID_ARG;
+  if (topk > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  return MISA_OK;
+}
+
+size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
+  const int64_t M = (L + B - 1) / B;
+  const int64_t nchunk = (M + kRouteChunk - 1) / kRouteChunk;
+  return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float));
+}
+size_t score_ws(int nseq, int T, int64_t L) {
+  return kStatusBytes + align256((size_t)nseq * T * L * sizeof(float));
+}
+size_t dagger_ws(int nseq, int T, int kprime) {
+  const size_t rows = (size_t)nseq * T;
+  return kStatusBytes + 2 * align256(rows * kprime * sizeof(int32_t)) +
+         align256(rows * sizeof(int32_t));
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws_bytes < need) return MISA_ERR_WORKSPACE_TOO_SMALL;
+  return check_dev(ws, need, 256);
+}
+
+int* status_word(void* ws) { return reinterpret_cast<int*>(ws); }
+char* ws_region(void* ws, size_t off) { return reinterpret_cast<char*>(ws) + kStatusBytes + off; }
+
+}  // namespace
+
+extern "C" {
+
+size_t misa_workspace_size(int op, int nseq, int T, int H, int d, int64_t L, int B, int h,
+                           int topk, int kprime) {
+  if (check_shape(nseq, T, H, d, L) != MISA_OK) return 0;
+  switch (op) {
+    case MISA_OP_ROUTE_HEADS:
+      if (B < 1 || h < 1 || h > H) return 0;
+      return route_ws(nseq, T, H, L, B);
+    case MISA_OP_SCORE_TOPK:
+      if (h < 1 || h > H || check_topk(topk) != MISA_OK) return 0;
+      return score_ws(nseq, T, L);
+    case MISA_OP_DSA_TOPK:
+      if (check_topk(topk) != MISA_OK) return 0;
+      return score_ws(nseq, T, L);
+    case MISA_OP_DAGGER_RERANK:
+      if (check_topk(topk) != MISA_OK || kprime < topk || kprime > MISA_MAX_TOPK) return 0;
+      return dagger_ws(nseq, T, kprime);
+    default:
+      return 0;
+  }
+}
+
+int misa_pool_keys(const uint16_t* k, int nseq, int64_t L, int d, int B, float* k_pool,
+                   void* stream) {
+  MISA_TRY(check_shape(nseq, 1, 1, d, L));
+  if (B < 1) return MISA_ERR_INVALID_ARG;
+  const int64_t M = (L + B - 1) / B;
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(k_pool, (size_t)nseq * M * d * 4, 16));
+  return cuda_status(launch_pool_mean(k, nseq, L, B, k_pool, (cudaStream_t)stream));
+}
+
+int misa_route_heads(const uint16_t* q, const float* w, const uint16_t* k, const float* k_pool,
+                     const int32_t* pos, int nseq, int T, int H, int d, int64_t L, int B, int h,
+                     int32_t* heads, float* E, void* ws, size_t ws_bytes, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  if (B < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)nseq * T;
+  const int64_t M = (L + B - 1) / B;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(k_pool, (size_t)nseq * M * d * 4, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  MISA_TRY(check_dev(heads, rows * h * 4, 4));
+  MISA_TRY(check_opt(E, rows * H * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, route_ws(nseq, T, H, L, B)));
+  const int nchunk = (int)((M + kRouteChunk - 1) / kRouteChunk);
+  return cuda_status(launch_route(q, w, k, k_pool, pos, nseq, T, H, L, B, h, heads, E,
+                                  reinterpret_cast<float*>(ws_region(ws, 0)), nchunk,
+                                  status_word(ws), (cudaStream_t)stream));
+}
+
+static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* k,
+                             const int32_t* heads, int h, const int32_t* pos, int nseq, int T,
+                             int H, int d, int64_t L, int topk, int32_t* idx, float* vals,
+                             float* scores, void* ws, size_t ws_bytes, void* stream) {
+  const size_t rows = (size_t)nseq * T;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  if (heads) MISA_TRY(check_dev(heads, rows * h * 4, 4));
+  MISA_TRY(check_dev(idx, rows * topk * 4, 4));
+  MISA_TRY(check_opt(vals, rows * topk * 4, 4));
+  MISA_TRY(check_opt(scores, rows * L * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, score_ws(nseq, T, L)));
+  cudaStream_t st = (cudaStream_t)stream;
+  float* sc = scores ? scores : reinterpret_cast<float*>(ws_region(ws, 0));
+  int* status = status_word(ws);
+  MISA_TRY(cuda_status(launch_score_simt(q, w, k, heads, h, pos, nullptr, nullptr, nseq, T, H,
+                                         L, sc, L, status, st)));
+  return cuda_status(launch_topk(sc, L, pos, L, nullptr, nullptr, (int)rows, topk, idx, vals,
+                                 status, st));
+}
+
+int misa_score_topk(const uint16_t* q, const float* w, const uint16_t* k, const int32_t* heads,
+                    const int32_t* pos, int nseq, int T, int H, int d, int64_t L, int h,
+                    int topk, int32_t* idx, float* vals, float* scores, void* ws,
+                    size_t ws_bytes, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  if (h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  if (h > MISA_MAX_ROUTED) return MISA_ERR_UNSUPPORTED;
+  MISA_TRY(check_topk(topk));
+  if (heads == nullptr) return MISA_ERR_INVALID_ARG;
+  return score_topk_common(q, w, k, heads, h, pos, nseq, T, H, d, L, topk, idx, vals, scores,
+                           ws, ws_bytes, stream);
+}
+
+int dsa_score_topk(const uint16_t* q, const float* w, const uint16_t* k, const int32_t* pos,
+                   int nseq, int T, int H, int d, int64_t L, int topk, int32_t* idx,
+                   float* vals, float* scores, void* ws, size_t ws_bytes, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  MISA_TRY(check_topk(topk));
+  return score_topk_common(q, w, k, nullptr, H, pos, nseq, T, H, d, L, topk, idx, vals, scores,
+                           ws, ws_bytes, stream);
+}
+
+int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k, const int32_t* pos,
+                       const int32_t* cand, int nseq, int T, int H, int d, int64_t L, int kprime,
+                       int topk, int32_t* idx, float* vals, void* ws, size_t ws_bytes,
+                       void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  MISA_TRY(check_topk(topk));
+  if (kprime < topk) return MISA_ERR_INVALID_ARG;
+  if (kprime > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)nseq * T;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  MISA_TRY(check_dev(cand, rows * kprime * 4, 4));
+  MISA_TRY(check_dev(idx, rows * topk * 4, 4));
+  MISA_TRY(check_opt(vals, rows * topk * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, dagger_ws(nseq, T, kprime)));
+  cudaStream_t st = (cudaStream_t)stream;
+  int* status = status_word(ws);
+  const size_t ids_bytes = align256(rows * kprime * sizeof(int32_t));
+  int32_t* sorted = reinterpret_cast<int32_t*>(ws_region(ws, 0));
+  float* cscore = reinterpret_cast<float*>(ws_region(ws, ids_bytes));
+  int32_t* count = reinterpret_cast<int32_t*>(ws_region(ws, 2 * ids_bytes));
+  MISA_TRY(cuda_status(
+      launch_sort_candidates(cand, pos, (int)rows, L, kprime, sorted, count, status, st)));
+  MISA_TRY(cuda_status(launch_score_simt(q, w, k, nullptr, H, pos, sorted, count, nseq, T, H, L,
+                                         cscore, kprime, status, st)));
+  return cuda_status(launch_topk(cscore, kprime, pos, L, count, sorted, (int)rows, topk, idx,
+                                 vals, status, st));
+}
+
+const char* misa_status_string(int status) {
+  switch (status) {
+    case MISA_OK: return "ok";
+    case MISA_ERR_INVALID_ARG: return "invalid argument";
+    case MISA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MISA_ERR_CUDA: return "CUDA error";
+    case MISA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MISA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MISA_ERR_BAD_DEVICE_INPUT: return "device input out of range (pos, head id or candidate)";
+    default: return "unknown status";
+  }
+}
+
+int misa_check_device_status(void* ws, void* stream) {
+  if (ws == nullptr) return MISA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MISA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MISA_ERR_CUDA;
+  if (v != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MISA_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Host-side launchers shared between the kernel files and the C ABI layer.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace misa {
+
+// Workspace layout helpers: every region starts on a 256-byte boundary.
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace header holding the sticky device status word.
+constexpr size_t kStatusBytes = 256;
+
+// Router: blocks of the prefix handled by one CTA of the partial-energy pass.
+constexpr int kRouteChunk = 32;
+
+// K1 -- mean pooling (pool.cu)
+cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, float* k_pool,
+                             cudaStream_t st);
+
+// K2 -- router: partial head energies per chunk of blocks, then E and top-h (route.cu)
+cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
+                         const float* k_pool, const int32_t* pos, int nseq, int T, int H,
+                         int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
+                         int nchunk, int* status, cudaStream_t st);
+
+// K4 -- token scoring on CUDA cores, any head subset (score_simt.cu).
+//   heads == nullptr: all H heads (dense, Eq. 1); otherwise hsel heads per row (Eq. 9).
+//   gather_ids != nullptr: score the tokens gather_ids[row, 0 .. gather_len[row]) instead
+//   of the prefix 0 .. pos[row]; output row stride is `out_stride`.
+cudaError_t launch_score_simt(const uint16_t* q, const float* w, const uint16_t* k,
+                              const int32_t* heads, int hsel, const int32_t* pos,
+                              const int32_t* gather_ids, const int32_t* gather_len,
+                              int nseq, int T, int H, int64_t L, float* out,
+                              int64_t out_stride, int* status, cudaStream_t st);
+
+// K5 -- per-row top-k selection (topk.cu).
+//   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.
+//   index_map (nullable, same stride) gives the token id of each entry; the entries of a
+//   row must then be in ascending token order (ties resolve by array order).
+cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
+                        const int32_t* gather_len, const int32_t* index_map, int rows,
+                        int topk, int32_t* idx, float* vals, int* status, cudaStream_t st);
+
+// Power-of-two length of the shared-memory sort buffer for `topk` entries (topk.cu).
+int topk_sort_size(int topk);
+
+// K7 -- MISA-dagger candidate preparation: sort each row's candidates ascending,
+// drop empty / out-of-prefix slots, count the valid ones (rerank.cu).
+cudaError_t launch_sort_candidates(const int32_t* cand, const int32_t* pos, int rows,
+                                   int64_t L, int kprime, int32_t* sorted, int32_t* count,
+                                   int* status, cudaStream_t st);
+
+}  // namespace misa

@@ -1,0 +1,75 @@
+// K1: block mean pooling of indexer keys -- Eq. (4) of the MISA paper summary
+// (Methodology section 1), with Pool read as the arithmetic mean of a block's keys.
+//
+// HBM-bound: every key is read once (256 B per token) and each pooled key (512 B
+// fp32) is written once.  One warp owns one (sequence, block): its two half-warps
+// walk the even and odd tokens of the block, each lane owning one 16-byte slice
+// (8 dims) of the 256-byte key row, so every warp-wide load covers two whole rows
+// (512 contiguous bytes).  Eight token pairs are loaded before any is accumulated to
+// keep enough bytes in flight per SM.
+#include "common.cuh"
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+__device__ __forceinline__ void acc8(float (&a)[8], const uint4& v) {
+  a[0] += bf16lo(v.x); a[1] += bf16hi(v.x);
+  a[2] += bf16lo(v.y); a[3] += bf16hi(v.y);
+  a[4] += bf16lo(v.z); a[5] += bf16hi(v.z);
+  a[6] += bf16lo(v.w); a[7] += bf16hi(v.w);
+}
+
+__global__ void __launch_bounds__(256) pool_mean_kernel(const uint4* __restrict__ k, int nseq,
+                                                        int64_t L, int B, int M,
+                                                        float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int half = lane >> 4;   // 0: even tokens of the block, 1: odd tokens
+  const int vec = lane & 15;    // which 16-byte slice of the key row
+  const int64_t items = (int64_t)nseq * M;
+  for (int64_t it = warp; it < items; it += nwarps) {
+    const int64_t n = it / M;
+    const int64_t b = it - n * M;
+    const int64_t s0 = b * B;
+    const int64_t s1 = min(s0 + (int64_t)B, L);
+    const uint4* base = k + n * L * 16 + vec;   // a key row is 16 uint4
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int64_t s = s0 + half;
+    for (; s + 14 < s1; s += 16) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcs(base + (s + 2 * u) * 16);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc8(a, v[u]);
+    }
+    for (; s < s1; s += 2) acc8(a, __ldcs(base + s * 16));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] += __shfl_down_sync(0xffffffffu, a[i], 16);
+    if (half == 0) {
+      const float inv = 1.0f / (float)(s1 - s0);
+      float4* o = reinterpret_cast<float4*>(out + it * kHeadDim + vec * 8);
+      o[0] = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
+      o[1] = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, float* k_pool,
+                             cudaStream_t st) {
+  const int M = (int)((L + B - 1) / B);
+  const int64_t items = (int64_t)nseq * M;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (items + 7) / 8;           // 8 warps per CTA
+  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  pool_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M,
+                                         k_pool);
+  return cudaGetLastError();
+}
+
+}  // namespace misa

@@ -1,0 +1,81 @@
+"""The C-ABI library on the host: it loads, exports every symbol include/misa.h
+declares, sizes workspaces, and rejects invalid arguments before touching the GPU.
+No compute call is made here (CPU only)."""
+
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "long_context_block_b200", "libmisa_b200.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from long_context_block_b200.build import build
+        build()
+    from long_context_block_b200 import _binding
+    return _binding
+
+
+def test_exports_every_declared_symbol(lib):
+    names = lib.declared_symbols()
+    assert {"misa_pool_keys", "misa_route_heads", "misa_score_topk", "dsa_score_topk",
+            "misa_dagger_rerank"} <= set(names)
+    cdll = ctypes.CDLL(LIB)
+    for n in names:
+        assert hasattr(cdll, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+
+
+def test_workspace_sizes(lib):
+    ws = lib.misa_workspace_size
+    # route: 256-byte header + rows * chunks * H fp32, chunk = 32 blocks
+    assert ws(1, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 16 * 64 * 4
+    assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4
+    assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4
+    assert ws(4, 16, 1, 64, 128, 131072, 64, 8, 2048, 8192) == 256 + 2 * 16 * 8192 * 4 + 256
+    # invalid sizes report 0
+    assert ws(1, 0, 1, 64, 128, 1024, 64, 8, 16, 16) == 0
+    assert ws(1, 1, 1, 64, 128, 1024, 64, 65, 16, 16) == 0
+    assert ws(2, 1, 1, 64, 64, 1024, 64, 8, 16, 16) == 0
+    assert ws(4, 1, 1, 64, 128, 1024, 64, 8, 32, 16) == 0
+    assert ws(9, 1, 1, 64, 128, 1024, 64, 8, 16, 16) == 0
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    c = lib.library()
+    null = None
+    # null pointers -> INVALID_ARG (1), before any CUDA call
+    assert c.misa_pool_keys(null, 1, 1024, 128, 64, null, null) == 1
+    # d != 128 -> UNSUPPORTED (2)
+    assert c.misa_pool_keys(null, 1, 1024, 64, 64, null, null) == 2
+    # B < 1
+    assert c.misa_pool_keys(null, 1, 1024, 128, 0, null, null) == 1
+    # h > H
+    assert c.misa_route_heads(null, null, null, null, null, 1, 1, 8, 128, 1024, 64, 9, null,
+                              null, null, 0, null) == 1
+    # h > 16 routed heads is not built
+    assert c.misa_score_topk(null, null, null, null, null, 1, 1, 64, 128, 1024, 17, 16, null,
+                             null, null, null, 0, null) == 2
+    # topk < 1, topk > 16384
+    assert c.dsa_score_topk(null, null, null, null, 1, 1, 64, 128, 1024, 0, null, null, null,
+                            null, 0, null) == 1
+    assert c.dsa_score_topk(null, null, null, null, 1, 1, 64, 128, 1024, 16385, null, null,
+                            null, null, 0, null) == 2
+    # k' < k
+    assert c.misa_dagger_rerank(null, null, null, null, null, 1, 1, 64, 128, 1024, 8, 16, null,
+                                null, null, 0, null) == 1
+    assert c.misa_check_device_status(null, null) == 1
+
+
+def test_status_strings(lib):
+    c = lib.library()
+    for code in range(0, 7):
+        assert c.misa_status_string(code)
+    assert c.misa_status_string(99) == b"unknown status"

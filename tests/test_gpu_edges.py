@@ -1,0 +1,132 @@
+"""Edge cases of the CUDA path against the fp64 oracle (GPU): ragged blocks, prefixes
+shorter than a block or than k, h = 1 and h = H, k' = k, ties, zero and negative
+weights, odd head counts, B = 1 and B > L, many rows, the largest k, bad device
+input, and guard bands around every output."""
+
+import numpy as np
+import pytest
+import torch
+
+from synth import Workload, fp32_to_bf16_bits, make_inputs
+from tests import gpu_path
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import long_context_block_b200 as M
+    return M
+
+
+def _wl(**kw):
+    base = dict(name="edge", nseq=2, T=5, L=300, H=8, d=128, h=3, B=64, topk=40, kprime=80,
+                pos_mode="tail", drift=True, needles=2)
+    base.update(kw)
+    return Workload(**base)
+
+
+def _random_pos(x, seed, lo=0):
+    rng = np.random.default_rng(seed)
+    x.pos = rng.integers(lo, x.wl.L, size=x.pos.shape).astype(np.int32)
+    return x
+
+
+CASES = {
+    "ragged_L_random_pos": dict(),
+    "prefix_shorter_than_block": dict(L=50, B=64, topk=16, kprime=32),
+    "prefix_shorter_than_k": dict(L=100, topk=256, kprime=512),
+    "h1": dict(h=1),
+    "h_equals_H": dict(h=8),
+    "kprime_equals_k": dict(kprime=40),
+    "H32_B128": dict(H=32, B=128, L=1000, h=8, topk=64, kprime=128),
+    "H3_odd": dict(H=3, h=2, L=257, B=16),
+    "H128_max_heads": dict(H=128, h=16, L=600, topk=100, kprime=200),
+    "B1": dict(B=1, L=200, topk=20, kprime=40),
+    "B_larger_than_L": dict(B=1024, L=300),
+    "many_rows": dict(nseq=3, T=150, L=700, topk=50, kprime=100),
+    "max_topk": dict(nseq=1, T=2, L=20000, topk=16384, kprime=16384, B=128),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_edge_case(M, case):
+    wl = _wl(**CASES[case])
+    x = make_inputs(wl, seed=11)
+    if case not in ("prefix_shorter_than_k", "max_topk"):
+        x = _random_pos(x, seed=5)
+    q, w, k, pos = gpu_path.to_device(x)
+    out = gpu_path.run_all(M, q, w, k, pos, wl.B, wl.h, wl.topk, wl.kprime)
+    rows = np.arange(wl.rows)
+    host = gpu_path.rows_to_host(out, rows, wl.T)
+    gpu_path.check_rows(x, host, rows, wl.B, wl.h, wl.topk, wl.kprime)
+
+
+def test_all_scores_tied_and_zero_weights(M):
+    """Keys all equal and every q.k negative: every score is exactly 0 and every E is 0,
+    so the selections must be the lowest indices (ties -> lower index)."""
+    wl = _wl(nseq=1, T=3, L=500, H=8, h=3, topk=64, kprime=128)
+    x = make_inputs(wl, seed=3)
+    kv = np.full((128,), 0.05, dtype=np.float32)
+    x.k_bits[:] = fp32_to_bf16_bits(kv)[None, None, :]
+    qv = -np.abs((x.q_bits.astype(np.uint32) << 16).view(np.float32))
+    x.q_bits = fp32_to_bf16_bits(qv)
+    x.w[:] = 0.0
+    x.w[0, 0, 2] = -1.5
+    q, w, k, pos = gpu_path.to_device(x)
+    out = gpu_path.run_all(M, q, w, k, pos, wl.B, wl.h, wl.topk, wl.kprime)
+    assert torch.all(out["heads"].cpu() == torch.arange(3, dtype=torch.int32))
+    for key in ("idx", "didx", "gidx"):
+        assert torch.all(out[key].cpu() == torch.arange(64, dtype=torch.int32)), key
+    assert torch.all(out["cand"].cpu() == torch.arange(128, dtype=torch.int32))
+
+
+def test_bad_device_input_is_reported_not_faulting(M):
+    """pos >= L and out-of-prefix candidates are clamped / skipped and reported through
+    the workspace status word."""
+    wl = _wl(nseq=1, T=2, L=256, topk=16, kprime=32)
+    x = make_inputs(wl, seed=4)
+    q, w, k, pos = gpu_path.to_device(x)
+    bad_pos = pos.clone()
+    bad_pos[0, 1] = 10_000
+    kp = M.misa_pool_keys(k, wl.B)
+    M.misa_route_heads(q, w, k, kp, bad_pos, wl.B, wl.h)
+    with pytest.raises(M.MisaError) as e:
+        M.misa_check_device_status(q.device)
+    assert e.value.status == 6
+    M.misa_check_device_status(q.device)  # cleared
+    cand = torch.full((1, 2, 32), -1, dtype=torch.int32, device=q.device)
+    cand[0, 0, 0] = 5
+    cand[0, 0, 1] = 100_000
+    idx, vals = M.misa_dagger_rerank(q, w, k, pos, cand, 16)
+    with pytest.raises(M.MisaError):
+        M.misa_check_device_status(q.device)
+    assert idx[0, 0, 0].item() == 5 and idx[0, 0, 1].item() == -1
+
+
+def test_guard_bands_untouched(M):
+    wl = _wl(nseq=2, T=3, L=400, topk=32, kprime=64)
+    x = make_inputs(wl, seed=9)
+    q, w, k, pos = gpu_path.to_device(x)
+    G = 1024
+    rows = wl.rows
+
+    def banded(n, dtype, fill):
+        buf = torch.full((n + 2 * G,), fill, dtype=dtype, device=q.device)
+        return buf, buf[G:G + n]
+
+    kp_buf, kp = banded(2 * 7 * 128, torch.float32, 7.0)
+    M.misa_pool_keys(k, wl.B, out=kp.view(2, 7, 128))
+    h_buf, heads = banded(rows * wl.h, torch.int32, 77)
+    e_buf, E = banded(rows * wl.H, torch.float32, 7.0)
+    M.misa_route_heads(q, w, k, kp.view(2, 7, 128), pos, wl.B, wl.h, return_E=True,
+                       heads=heads.view(2, 3, wl.h), E=E.view(2, 3, wl.H))
+    i_buf, idx = banded(rows * wl.topk, torch.int32, 77)
+    v_buf, vals = banded(rows * wl.topk, torch.float32, 7.0)
+    M.misa_score_topk(q, w, k, heads.view(2, 3, wl.h), pos, wl.topk,
+                      idx=idx.view(2, 3, wl.topk), vals=vals.view(2, 3, wl.topk))
+    torch.cuda.synchronize()
+    for buf, fill in ((kp_buf, 7.0), (h_buf, 77), (e_buf, 7.0), (i_buf, 77), (v_buf, 7.0)):
+        assert torch.all(buf[:G] == fill) and torch.all(buf[-G:] == fill)

@@ -64,10 +64,10 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str, tag: int):
+        self.gpu = gpu_id            # nvidia-smi --id value (the device UUID)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{tag}.csv")
 
     def __enter__(self):
         try:
@@ -75,8 +75,9 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.STDOUT)
+            time.sleep(0.5)
         except Exception:
             self.proc = None
         return self
@@ -170,14 +171,16 @@ def run_reference(args, wl):
     return 0
 
 
-def cpu_baseline(wl, budget_s: float = 12.0):
-    """Time the oracle's MISA path on the host cores over as many rows as fit the budget."""
+def cpu_baseline(wl, budget_s: float = 10.0):
+    """Time the oracle's MISA path on the host cores: passes over the workload's query
+    rows until the time budget is used (at least one row)."""
     import oracle.misa_oracle as orc
     from threadpoolctl import threadpool_info
-    x = make_inputs(wl.replace(nseq=min(wl.nseq, 8)) if wl.T == 1 else wl, seed=0)
+    x = make_inputs(wl, seed=0)
     units, rows_done = 0, 0
     t0 = time.perf_counter()
-    for row in range(x.wl.rows):
+    for it in range(1 << 30):
+        row = it % x.wl.rows
         n, t = divmod(row, x.wl.T)
         k = orc.bf16_bits_to_f64(x.k_bits[n])
         q_t = orc.bf16_bits_to_f64(x.q_bits[n, t])
@@ -259,9 +262,18 @@ def run_cuda(args, wl):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def timed(step_fn, steps, warmup, **kw):
+    def timed(step_fn, steps, warmup, load_s=0.0, **kw):
         for i in range(warmup):
             step_fn(i)
+        if load_s > 0:   # untimed steady-state load so the clock sampler sees this kernel mix
+            torch.cuda.synchronize()
+            t_end = time.perf_counter() + load_s
+            i = warmup
+            while time.perf_counter() < t_end:
+                for _ in range(50):
+                    step_fn(i)
+                    i += 1
+                torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -276,8 +288,9 @@ def run_cuda(args, wl):
             ms = float(t.item())
         return ms / steps
 
-    with ClockSampler(local) as clk:
-        ms_misa = timed(misa_step, args.steps, args.warmup, record=True)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid, rank) as clk:
+        ms_misa = timed(misa_step, args.steps, args.warmup, load_s=2.0, record=True)
     clocks = clk.summary()
     M.misa_check_device_status(dev)
     score_ms = [a.elapsed_time(b) for a, b in ev_score]

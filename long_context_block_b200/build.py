@@ -1,6 +1,7 @@
 """Build the MISA indexer shared library (libmisa_b200.so) in-tree for sm_100a.
 
-    python -m long_context_block_b200.build        # or: from long_context_block_b200.build import build
+    python long_context_block_b200/build.py [-f] [-v] [--ptxas]
+    (or __graft_entry__.build(); importing the package needs the built library)
 
 Each CUDA source is compiled to an object under _build/ (in parallel), then linked
 into long_context_block_b200/libmisa_b200.so.  The CUDA runtime is linked

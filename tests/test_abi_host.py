@@ -14,9 +14,8 @@ LIB = os.path.join(ROOT, "long_context_block_b200", "libmisa_b200.so")
 
 @pytest.fixture(scope="module")
 def lib():
-    if not os.path.exists(LIB):
-        from long_context_block_b200.build import build
-        build()
+    import __graft_entry__
+    __graft_entry__.build()
     from long_context_block_b200 import _binding
     return _binding
 

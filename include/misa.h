@@ -62,6 +62,8 @@ extern "C" {
 #define MISA_ERR_DEVICE_TIMEOUT      4  /* a bounded device-side wait expired            */
 #define MISA_ERR_WORKSPACE_TOO_SMALL 5  /* ws_bytes < misa_workspace_size(...)            */
 #define MISA_ERR_BAD_DEVICE_INPUT    6  /* device data out of range (pos >= L, cand)     */
+#define MISA_ERR_STATIC_SCRATCH_TOO_SMALL 7  /* call larger than the fixed scratch of
+                                                misa_score_topk_noalloc                 */
 
 /* Operation ids for misa_workspace_size. */
 #define MISA_OP_ROUTE_HEADS   1
@@ -141,6 +143,30 @@ int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k,
                        const int32_t* pos, const int32_t* cand, int nseq, int T, int H,
                        int d, int64_t L, int kprime, int topk, int32_t* idx, float* vals,
                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * misa_score_topk without any allocation or workspace.  The paper has no
+ * counterpart of this entry point; it serves callers that cannot allocate device
+ * memory or pass a workspace (code running inside an allocator-free region of a
+ * serving engine, or a plugin whose host framework owns every allocation).
+ *
+ * Computes exactly what misa_score_topk computes (Ihat and its top-k; vals may be
+ * NULL).  Its scratch is a fixed array inside the library's device image: 16 MiB
+ * on every GPU that loads the library, held until the process exits, enough for
+ * nseq * T * L <= 4,194,304 scores; larger calls return
+ * MISA_ERR_STATIC_SCRATCH_TOO_SMALL and enqueue nothing.  All calls on a device
+ * share that array and it keeps the last call's contents, so calls whose GPU work
+ * overlaps (other streams, other host threads) race and must be serialised by the
+ * caller.  The first call on each device looks up the array's address with that
+ * device current; make it before any stream capture.  device_status (nullable,
+ * device int32) receives this call's device-side status word (MISA_OK or
+ * MISA_ERR_BAD_DEVICE_INPUT), as misa_check_device_status would report it.
+ * Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+int misa_score_topk_noalloc(const uint16_t* q, const float* w, const uint16_t* k,
+                            const int32_t* heads, const int32_t* pos, int nseq, int T, int H,
+                            int d, int64_t L, int h, int topk, int32_t* idx, float* vals,
+                            int32_t* device_status, void* stream);
 
 /* Static text for a status code.  Host-only. */
 const char* misa_status_string(int status);

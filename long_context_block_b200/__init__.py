@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     misa_pool_keys,
     misa_route_heads,
     misa_score_topk,
+    misa_score_topk_noalloc,
     misa_workspace_size,
     workspace,
 )

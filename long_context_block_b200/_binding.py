@@ -22,7 +22,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "misa.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m long_context_block_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python long_context_block_b200/build.py` "
         "(or __graft_entry__.build()); this package has no fallback path")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -41,6 +41,8 @@ _SIGS = {
                                 _p, _p, _p, _p, _c_sz, _p]),
     "misa_dagger_rerank": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_i64,
                                     _c_int, _c_int, _p, _p, _p, _c_sz, _p]),
+    "misa_score_topk_noalloc": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
+                                         _c_i64, _c_int, _c_int, _p, _p, _p, _p]),
     "misa_status_string": (ctypes.c_char_p, [_c_int]),
     "misa_check_device_status": (_c_int, [_p, _p]),
 }
@@ -245,4 +247,26 @@ def misa_dagger_rerank(q, w, k, pos, cand, topk: int, return_vals: bool = True, 
            _lib.misa_dagger_rerank(_ptr(q), _ptr(w), _ptr(k), _ptr(pos), _ptr(cand), nseq, T, H,
                                    d, L, kprime, topk, _ptr(idx), _ptr(vals), _ptr(ws),
                                    ws.numel(), _stream()))
+    return (idx, vals) if return_vals else idx
+
+
+def misa_score_topk_noalloc(q, w, k, heads, pos, topk: int, return_vals: bool = True, idx=None,
+                            vals=None, device_status=None):
+    """misa_score_topk for callers that cannot allocate: the library uses its own fixed
+    16 MiB scratch (nseq * T * L <= 4,194,304) instead of a workspace.  Outputs are
+    allocated here only when not passed in; pass idx / vals / device_status to make
+    the call allocation-free from Python too.  Calls whose GPU work overlaps race on
+    the shared scratch and must be serialised."""
+    q, k = _bits(q, "q"), _bits(k, "k")
+    w = _dev(w, "w", torch.float32)
+    heads = _dev(heads, "heads", torch.int32)
+    pos = _dev(pos, "pos", torch.int32)
+    nseq, T, H, d = q.shape
+    L = k.shape[1]
+    h = heads.shape[-1]
+    idx, vals = _outs((nseq, T), topk, q.device, idx, vals, return_vals)
+    _check("misa_score_topk_noalloc",
+           _lib.misa_score_topk_noalloc(_ptr(q), _ptr(w), _ptr(k), _ptr(heads), _ptr(pos), nseq,
+                                        T, H, d, L, h, topk, _ptr(idx), _ptr(vals),
+                                        _ptr(device_status), _stream()))
     return (idx, vals) if return_vals else idx

@@ -242,6 +242,8 @@ const char* misa_status_string(int status) {
     case MISA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case MISA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case MISA_ERR_BAD_DEVICE_INPUT: return "device input out of range (pos, head id or candidate)";
+    case MISA_ERR_STATIC_SCRATCH_TOO_SMALL:
+      return "call exceeds the fixed scratch of misa_score_topk_noalloc (nseq*T*L > 4194304)";
     default: return "unknown status";
   }
 }

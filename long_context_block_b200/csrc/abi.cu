@@ -84,8 +84,9 @@ size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
   const int64_t nchunk = (M + kRouteChunk - 1) / kRouteChunk;
   return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float));
 }
-size_t score_ws(int nseq, int T, int64_t L) {
-  return kStatusBytes + align256((size_t)nseq * T * L * sizeof(float));
+size_t score_ws(int nseq, int T, int64_t L, int nh) {
+  return kStatusBytes + align256((size_t)nseq * T * L * sizeof(float)) +
+         score_tc_ws_bytes((int64_t)nseq * T, nh);
 }
 size_t dagger_ws(int nseq, int T, int kprime) {
   const size_t rows = (size_t)nseq * T;
@@ -114,10 +115,10 @@ size_t misa_workspace_size(int op, int nseq, int T, int H, int d, int64_t L, int
       return route_ws(nseq, T, H, L, B);
     case MISA_OP_SCORE_TOPK:
       if (h < 1 || h > H || check_topk(topk) != MISA_OK) return 0;
-      return score_ws(nseq, T, L);
+      return score_ws(nseq, T, L, h);
     case MISA_OP_DSA_TOPK:
       if (check_topk(topk) != MISA_OK) return 0;
-      return score_ws(nseq, T, L);
+      return score_ws(nseq, T, L, H);
     case MISA_OP_DAGGER_RERANK:
       if (check_topk(topk) != MISA_OK || kprime < topk || kprime > MISA_MAX_TOPK) return 0;
       return dagger_ws(nseq, T, kprime);
@@ -170,12 +171,19 @@ static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* 
   MISA_TRY(check_dev(idx, rows * topk * 4, 4));
   MISA_TRY(check_opt(vals, rows * topk * 4, 4));
   MISA_TRY(check_opt(scores, rows * L * 4, 4));
-  MISA_TRY(check_ws(ws, ws_bytes, score_ws(nseq, T, L)));
+  const int nh = heads ? h : H;
+  MISA_TRY(check_ws(ws, ws_bytes, score_ws(nseq, T, L, nh)));
   cudaStream_t st = (cudaStream_t)stream;
   float* sc = scores ? scores : reinterpret_cast<float*>(ws_region(ws, 0));
   int* status = status_word(ws);
-  MISA_TRY(cuda_status(launch_score_simt(q, w, k, heads, h, pos, nullptr, nullptr, nseq, T, H,
-                                         L, sc, L, status, st)));
+  if (score_tc_supported(nseq, T, nh, L)) {
+    void* tc_scratch = ws_region(ws, align256(rows * L * sizeof(float)));
+    MISA_TRY(cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, sc, L, tc_scratch,
+                                         status, st)));
+  } else {
+    MISA_TRY(cuda_status(launch_score_simt(q, w, k, heads, h, pos, nullptr, nullptr, nseq, T, H,
+                                           L, sc, L, status, st)));
+  }
   return cuda_status(launch_topk(sc, L, pos, L, nullptr, nullptr, (int)rows, topk, idx, vals,
                                  status, st));
 }

@@ -36,6 +36,16 @@ cudaError_t launch_score_simt(const uint16_t* q, const float* w, const uint16_t*
                               int nseq, int T, int H, int64_t L, float* out,
                               int64_t out_stride, int* status, cudaStream_t st);
 
+// K4 -- token scoring on tcgen05 tensor cores, rows streaming their own key prefix
+// (score_tc.cu).  Same contract as launch_score_simt without the gather mode; needs
+// score_tc_ws_bytes(rows, nh) bytes of 256-aligned scratch.
+bool score_tc_supported(int nseq, int T, int nh, int64_t L);
+size_t score_tc_ws_bytes(int64_t rows, int nh);
+cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
+                            const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
+                            int H, int64_t L, float* out, int64_t out_stride, void* scratch,
+                            int* status, cudaStream_t st);
+
 // K5 -- per-row top-k selection (topk.cu).
 //   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.
 //   index_map (nullable, same stride) gives the token id of each entry; the entries of a

@@ -232,19 +232,23 @@ def run_cuda(args, wl):
     units = wl.query_prefix_tokens()
     stream = torch.cuda.current_stream()
 
-    ev_score = []   # (start, end) around the routed score + top-k call
+    ev_calls = []   # per timed step: events around pool, route, routed score + top-k
 
     def misa_step(i, record=False):
         q, w, k, pos = sets[i % 2]
+        if record:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
         M.misa_pool_keys(k, wl.B, out=kp[i % 2])
+        if record:
+            ev[1].record(stream)
         M.misa_route_heads(q, w, k, kp[i % 2], pos, wl.B, wl.h, heads=heads)
         if record:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+            ev[2].record(stream)
         M.misa_score_topk(q, w, k, heads, pos, wl.topk, idx=idx, vals=vals)
         if record:
-            b.record(stream)
-            ev_score.append((a, b))
+            ev[3].record(stream)
+            ev_calls.append(ev)
 
     def dagger_step(i):
         q, w, k, pos = sets[i % 2]
@@ -293,8 +297,9 @@ def run_cuda(args, wl):
         ms_misa = timed(misa_step, args.steps, args.warmup, load_s=2.0, record=True)
     clocks = clk.summary()
     M.misa_check_device_status(dev)
-    score_ms = [a.elapsed_time(b) for a, b in ev_score]
-    score_ms_avg = sum(score_ms) / len(score_ms)
+    per_call = [[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in ev_calls]
+    call_ms = [sum(c[j] for c in per_call) / len(per_call) for j in range(3)]
+    score_ms_avg = call_ms[2]
     ms_dagger = timed(dagger_step, args.steps, args.warmup)
     ms_dsa = timed(dsa_step, args.steps, args.warmup)
     M.misa_check_device_status(dev)
@@ -339,7 +344,8 @@ def run_cuda(args, wl):
                      "peak_source": peaks["source"], "algorithmic_bytes": score_bytes,
                      "avg_ms": score_ms_avg},
         "paths": {
-            "misa": {"value": units * world / (ms_misa * 1e-3), "ms_per_step": ms_misa},
+            "misa": {"value": units * world / (ms_misa * 1e-3), "ms_per_step": ms_misa,
+                     "ms_pool": call_ms[0], "ms_route": call_ms[1], "ms_score_topk": call_ms[2]},
             "dsa": {"value": units * world / (ms_dsa * 1e-3), "ms_per_step": ms_dsa},
             "misa_dagger": {"value": units * world / (ms_dagger * 1e-3), "ms_per_step": ms_dagger},
             "speedup_misa_vs_dsa": ms_dsa / ms_misa,

@@ -82,11 +82,24 @@ int check_topk(int topk) {
 size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
   const int64_t M = (L + B - 1) / B;
   const int64_t nchunk = (M + kRouteChunk - 1) / kRouteChunk;
-  return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float));
+  return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float)) +
+         align256((size_t)nseq * T * sizeof(int));
 }
+// Rows up to this count whose length reaches kHistPathMinLen use the histogram-filtered
+// top-k, fed by a score histogram built in the tensor-core scorer's epilogue.
+constexpr int kHistPathMaxRows = 1024;
+constexpr int64_t kHistPathMinLen = 8192;
+
+bool hist_path(int nseq, int T, int64_t L) {
+  return (int64_t)nseq * T <= kHistPathMaxRows && L >= kHistPathMinLen;
+}
+
+size_t hist_path_bytes(int64_t rows) { return topk_hist_ws_bytes(rows); }
+
 size_t score_ws(int nseq, int T, int64_t L, int nh) {
-  return kStatusBytes + align256((size_t)nseq * T * L * sizeof(float)) +
-         score_tc_ws_bytes((int64_t)nseq * T, nh);
+  const int64_t rows = (int64_t)nseq * T;
+  return kStatusBytes + align256((size_t)rows * L * sizeof(float)) + score_tc_ws_bytes(rows, nh) +
+         (hist_path(nseq, T, L) ? hist_path_bytes(rows) : 0);
 }
 size_t dagger_ws(int nseq, int T, int kprime) {
   const size_t rows = (size_t)nseq * T;
@@ -153,8 +166,10 @@ int misa_route_heads(const uint16_t* q, const float* w, const uint16_t* k, const
   MISA_TRY(check_opt(E, rows * H * 4, 4));
   MISA_TRY(check_ws(ws, ws_bytes, route_ws(nseq, T, H, L, B)));
   const int nchunk = (int)((M + kRouteChunk - 1) / kRouteChunk);
+  const size_t part_bytes = align256(rows * nchunk * H * sizeof(float));
   return cuda_status(launch_route(q, w, k, k_pool, pos, nseq, T, H, L, B, h, heads, E,
                                   reinterpret_cast<float*>(ws_region(ws, 0)), nchunk,
+                                  reinterpret_cast<int*>(ws_region(ws, part_bytes)),
                                   status_word(ws), (cudaStream_t)stream));
 }
 
@@ -177,9 +192,23 @@ static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* 
   float* sc = scores ? scores : reinterpret_cast<float*>(ws_region(ws, 0));
   int* status = status_word(ws);
   if (score_tc_supported(nseq, T, nh, L)) {
-    void* tc_scratch = ws_region(ws, align256(rows * L * sizeof(float)));
+    const size_t sc_bytes = align256(rows * L * sizeof(float));
+    void* tc_scratch = ws_region(ws, sc_bytes);
+    if (hist_path(nseq, T, L)) {
+      char* hp = ws_region(ws, sc_bytes + score_tc_ws_bytes(rows, nh));
+      const size_t hb = align256(rows * kScoreHistBins * 4);
+      const size_t gb = align256(rows * 16 * 4);
+      uint32_t* hist = reinterpret_cast<uint32_t*>(hp);
+      uint32_t* gcount = reinterpret_cast<uint32_t*>(hp + hb);
+      uint64_t* cand = reinterpret_cast<uint64_t*>(hp + hb + gb);
+      MISA_TRY(cuda_status(cudaMemsetAsync(hist, 0, hb + gb, st)));
+      MISA_TRY(cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, sc, L,
+                                           tc_scratch, status, hist, st)));
+      return cuda_status(launch_topk_hist(sc, L, pos, L, hist, cand, gcount, (int)rows, topk, idx,
+                                          vals, st));
+    }
     MISA_TRY(cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, sc, L, tc_scratch,
-                                         status, st)));
+                                         status, nullptr, st)));
   } else {
     MISA_TRY(cuda_status(launch_score_simt(q, w, k, heads, h, pos, nullptr, nullptr, nseq, T, H,
                                            L, sc, L, status, st)));

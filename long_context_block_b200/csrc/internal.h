@@ -13,6 +13,13 @@ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Workspace header holding the sticky device status word.
 constexpr size_t kStatusBytes = 256;
 
+// Histogram of the top kScoreHistBits bits of the order-preserving score keys, used to
+// cut long rows down to a small candidate set before the exact top-k.
+constexpr int kScoreHistBits = 12;
+constexpr int kScoreHistBins = 1 << kScoreHistBits;
+// Candidate capacity per row of the histogram-filtered top-k.
+constexpr int kTopkCandCap = 16384;
+
 // Router: blocks of the prefix handled by one CTA of the partial-energy pass.
 constexpr int kRouteChunk = 32;
 
@@ -20,11 +27,12 @@ constexpr int kRouteChunk = 32;
 cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, float* k_pool,
                              cudaStream_t st);
 
-// K2 -- router: partial head energies per chunk of blocks, then E and top-h (route.cu)
+// K2 -- router: partial head energies per chunk of blocks, then E and top-h by the
+// last CTA of each row (route.cu).  `counters` is rows ints of scratch (zeroed here).
 cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
                          const float* k_pool, const int32_t* pos, int nseq, int T, int H,
                          int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
-                         int nchunk, int* status, cudaStream_t st);
+                         int nchunk, int* counters, int* status, cudaStream_t st);
 
 // K4 -- token scoring on CUDA cores, any head subset (score_simt.cu).
 //   heads == nullptr: all H heads (dense, Eq. 1); otherwise hsel heads per row (Eq. 9).
@@ -41,10 +49,12 @@ cudaError_t launch_score_simt(const uint16_t* q, const float* w, const uint16_t*
 // score_tc_ws_bytes(rows, nh) bytes of 256-aligned scratch.
 bool score_tc_supported(int nseq, int T, int nh, int64_t L);
 size_t score_tc_ws_bytes(int64_t rows, int nh);
+//   hist (nullable, zeroed by the caller): per-row kScoreHistBins-bin histogram of the
+//   written scores' keys, accumulated in the epilogue.
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
-                            int* status, cudaStream_t st);
+                            int* status, uint32_t* hist, cudaStream_t st);
 
 // K5 -- per-row top-k selection (topk.cu).
 //   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.
@@ -53,6 +63,17 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
 cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
                         const int32_t* gather_len, const int32_t* index_map, int rows,
                         int topk, int32_t* idx, float* vals, int* status, cudaStream_t st);
+
+// K5 for long rows with a histogram of their scores (topk.cu): the bins at or above the
+// bin of the row's k-th largest score are split into groups of output positions; a
+// scatter pass appends every candidate to its group's buffer and one CTA per group sorts
+// and writes it.  hist: rows x kScoreHistBins (filled by the scorer); gcount: rows x 16
+// (zeroed by the caller, directly after hist); cand: topk_hist_ws_bytes layout.
+cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
+                             const uint32_t* hist, uint64_t* cand, uint32_t* gcount, int rows,
+                             int topk, int32_t* idx, float* vals, cudaStream_t st);
+// Scratch of the histogram path: histogram, group counts, group buffers (256-aligned each).
+size_t topk_hist_ws_bytes(int64_t rows);
 
 // Power-of-two length of the shared-memory sort buffer for `topk` entries (topk.cu).
 int topk_sort_size(int topk);

@@ -4,29 +4,34 @@
 // the ordinary index-order pass, each row's candidates are first sorted ascending.
 // Empty slots (-1) and ids outside the query's prefix are dropped (the latter are
 // recorded as bad device input); `count` receives the number of valid candidates.
+#include "blocksort.cuh"
 #include "common.cuh"
 #include "internal.h"
 
 namespace misa {
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = kSortThreads;
 
 __global__ void __launch_bounds__(kThreads) sort_candidates_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pos, int64_t L, int kprime,
     int sortn, int32_t* __restrict__ sorted, int32_t* __restrict__ count, int* status,
     int64_t row0) {
-  extern __shared__ uint32_t buf[];   // [sortn]
+  extern __shared__ uint64_t buf[];   // [sortn]
   const int tid = threadIdx.x;
   const int64_t row = row0 + blockIdx.x;
   const int P = prefix_len(pos, row, L, tid == 0 ? status : nullptr);
+  __shared__ int s_count;
+  if (tid == 0) s_count = 0;
+  __syncthreads();
   int valid_local = 0;
+  // ascending token order = descending order of the complemented id; empty slots are 0
   for (int i = tid; i < sortn; i += kThreads) {
-    uint32_t v = 0xffffffffu;
+    uint64_t v = 0;
     if (i < kprime) {
       const int32_t c = cand[row * kprime + i];
       if (c >= 0 && c < P) {
-        v = (uint32_t)c;
+        v = (uint64_t)(~(uint32_t)c) << 32;
         ++valid_local;
       } else if (c != -1) {
         set_status(status, MISA_ERR_BAD_DEVICE_INPUT);
@@ -34,26 +39,12 @@ __global__ void __launch_bounds__(kThreads) sort_candidates_kernel(
     }
     buf[i] = v;
   }
-  // count valid entries (a thread may own several)
-  __shared__ int s_count;
-  if (tid == 0) s_count = 0;
-  __syncthreads();
   if (valid_local) atomicAdd(&s_count, valid_local);
-  // bitonic sort, ascending (invalid = 0xffffffff go last)
-  for (int kk = 2; kk <= sortn; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      __syncthreads();
-      for (int i = tid; i < (sortn >> 1); i += kThreads) {
-        const int lo = ((i & ~(j - 1)) << 1) | (i & (j - 1));
-        const int hi = lo | j;
-        const uint32_t a = buf[lo], b = buf[hi];
-        const bool asc = (lo & kk) == 0;
-        if (asc ? (a > b) : (a < b)) { buf[lo] = b; buf[hi] = a; }
-      }
-    }
+  sort_buf_desc(buf, sortn);
+  for (int i = tid; i < kprime; i += kThreads) {
+    const uint64_t v = buf[i];
+    sorted[row * kprime + i] = v ? (int32_t)(~(uint32_t)(v >> 32)) : -1;
   }
-  __syncthreads();
-  for (int i = tid; i < kprime; i += kThreads) sorted[row * kprime + i] = (int32_t)buf[i];
   if (tid == 0) count[row] = s_count;
 }
 
@@ -63,7 +54,7 @@ cudaError_t launch_sort_candidates(const int32_t* cand, const int32_t* pos, int 
                                    int64_t L, int kprime, int32_t* sorted, int32_t* count,
                                    int* status, cudaStream_t st) {
   const int sortn = topk_sort_size(kprime);
-  const size_t smem = (size_t)sortn * sizeof(uint32_t);
+  const size_t smem = (size_t)sortn * sizeof(uint64_t);
   cudaError_t e = cudaFuncSetAttribute(sort_candidates_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -54,7 +54,8 @@ struct DecodeCfg {
   // full[S], empty[S], qfull[2], qempty[2], accfull[A], accempty[A], drain
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
   static constexpr int kMiscBase = kBarBase + kNumBars * 8;
-  static constexpr int kSmemBytes = kMiscBase + 16 + 1024;   // + alignment slack
+  static constexpr int kHistBase = kMiscBase + 16;            // [kScoreHistBins] u32
+  static constexpr int kSmemBytes = kHistBase + kScoreHistBins * 4 + 1024;   // + alignment slack
   static_assert(N % 16 == 0 && N >= 16 && N <= 128, "N");
   static_assert(kQHalf % 1024 == 0, "q half tile must keep the 1 KB swizzle alignment");
 };
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ wsel, const int32_t* __restrict__ pos,
     const int32_t* __restrict__ tile_off, int rows, int T, int64_t L, float* __restrict__ out,
-    int64_t out_stride, int* status) {
+    int64_t out_stride, int* status, uint32_t* __restrict__ hist) {
   using C = DecodeCfg<N>;
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -126,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
   uint64_t* drain = accempty + C::kAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::kMiscBase);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + C::kMiscBase + 4);
+  uint32_t* shist = reinterpret_cast<uint32_t*>(base + C::kHistBase);
+  if (hist)
+    for (int b = tid; b < kScoreHistBins; b += kThreads) shist[b] = 0;
 
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -235,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;   // TMEM lanes this warp may read
     const int key_in_tile = quarter * 32 + lane;
+    const int etid = tid - 64;      // 0..127 over the four epilogue warps
     int acc_it = 0;
     int r = r_first;
     Seg sg;
@@ -265,8 +270,23 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
         tc_fence_before();
         mbar_arrive(&accempty[acc]);
         const int s = j * kTileKeys + key_in_tile;
-        if (s < P) orow[s] = sc;
+        if (s < P) {
+          orow[s] = sc;
+          if (hist) atomicAdd(&shist[score_key(sc) >> (32 - kScoreHistBits)], 1u);
+        }
         ++acc_it;
+      }
+      if (hist) {
+        // flush this row's histogram; the four epilogue warps are always in the same
+        // segment here, and leave together (the abort flag is read after the barrier)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        uint32_t* gh = hist + (int64_t)sg.r * kScoreHistBins;
+        for (int b = etid; b < kScoreHistBins; b += 128) {
+          const uint32_t v = shist[b];
+          if (v) { atomicAdd(gh + b, v); shist[b] = 0; }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        ok = *abort_flag == 0;
       }
     }
     __syncthreads();   // (A)
@@ -376,7 +396,8 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t nrows, uint32_t box_rows
 template <int N>
 cudaError_t launch_n(const CUtensorMap& tk, const CUtensorMap& tq, const float* wg,
                      const int32_t* pos, const int32_t* tile_off, int rows, int T, int64_t L,
-                     float* out, int64_t out_stride, int* status, cudaStream_t st) {
+                     float* out, int64_t out_stride, int* status, uint32_t* hist,
+                     cudaStream_t st) {
   using C = DecodeCfg<N>;
   cudaError_t e = cudaFuncSetAttribute(score_tc_decode_kernel<N>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -385,7 +406,7 @@ cudaError_t launch_n(const CUtensorMap& tk, const CUtensorMap& tq, const float* 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   score_tc_decode_kernel<N><<<sms, kThreads, C::kSmemBytes, st>>>(
-      tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status);
+      tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist);
   return cudaGetLastError();
 }
 
@@ -409,7 +430,7 @@ bool score_tc_supported(int nseq, int T, int nh, int64_t L) {
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
-                            int* status, cudaStream_t st) {
+                            int* status, uint32_t* hist, cudaStream_t st) {
   const int rows = nseq * T;
   const int nh = heads ? hsel : H;
   const int N = score_tc_padded_heads(nh);
@@ -429,14 +450,14 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
       !make_map(&tq, qg, (uint64_t)rows * N, (uint32_t)N))
     return cudaErrorInvalidValue;
   switch (N) {
-    case 16: return launch_n<16>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 32: return launch_n<32>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 48: return launch_n<48>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 64: return launch_n<64>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 80: return launch_n<80>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 96: return launch_n<96>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 112: return launch_n<112>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
-    case 128: return launch_n<128>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, st);
+    case 16: return launch_n<16>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 32: return launch_n<32>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 48: return launch_n<48>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 64: return launch_n<64>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 80: return launch_n<80>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 96: return launch_n<96>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 112: return launch_n<112>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
+    case 128: return launch_n<128>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -2,14 +2,28 @@
 // paper summary.  Output order: descending score, equal scores by ascending token
 // index; rows shorter than k are padded with index -1 and value -inf.
 //
-// One CTA (1024 threads) per row.  Scores are mapped to order-preserving uint32 keys
-// and the k-th largest key is found exactly by a three-pass radix select (11, 11 and
-// 10 bits; shared-memory histograms, a block-wide suffix scan picks the bin).  A
-// final pass in index order gathers every key above that threshold plus the lowest-
-// index keys equal to it, so that exactly k (key, index) pairs remain; a bitonic sort
-// of those 64-bit pairs in shared memory produces the output order.
+// Scores are mapped to order-preserving uint32 keys and the k-th largest key is found
+// exactly by a three-pass radix select (11, 11 and 10 bits; histograms in shared
+// memory, a block-wide suffix scan picks the bin).  A final pass in index order takes
+// every key above that threshold plus the lowest-index keys equal to it, so exactly k
+// (key, index) pairs remain; a bitonic sort of those 64-bit pairs in shared memory
+// gives the output order.
+//
+// topk_cluster_kernel (main form): a row is split over a thread-block cluster of G CTAs
+// (G = 1, 2, 4 or 8).  Each CTA reads its slice of the row from global memory once and
+// keeps it in shared memory as keys; the per-pass histograms are summed across the
+// cluster through distributed shared memory, so every CTA picks the same digit, and
+// the selected pairs are written straight into the leader CTA's sort buffer.
+// topk_kernel (fallback for rows too long for a cluster's shared memory): one CTA per
+// row, every pass re-reads the row from global memory.
+#include <cooperative_groups.h>
+
+#include "blocksort.cuh"
 #include "common.cuh"
+#include "groupsort.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace misa {
 namespace {
@@ -49,20 +63,31 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
   return base + incl - v;
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(
-    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
-    const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
-    int sortn, int32_t* __restrict__ idx, float* __restrict__ vals, int64_t row0) {
-  extern __shared__ uint64_t sel[];   // [sortn]
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t s_digit, s_above, s_cnt;
-  const int tid = threadIdx.x;
-  const int64_t row = row0 + blockIdx.x;
-  const int n = gather_len ? gather_len[row] : prefix_len(pos, row, L, nullptr);
-  const float* x = scores + row * stride;
-  const int32_t* imap = index_map ? index_map + row * stride : nullptr;
+// Write the first min(n, topk) sorted pairs of `sel` as (index, value), pad the rest.
+__device__ __forceinline__ void write_row(const uint64_t* sel, int n, int topk, int64_t row,
+                                          int32_t* idx, float* vals) {
+  const int nvalid = n < topk ? n : topk;
+  for (int i = threadIdx.x; i < topk; i += kThreads) {
+    const int64_t o = row * topk + i;
+    if (i < nvalid) {
+      const uint64_t v = sel[i];
+      idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
+      if (vals) vals[o] = key_score((uint32_t)(v >> 32));
+    } else {
+      idx[o] = -1;
+      if (vals) vals[o] = __int_as_float(0xff800000);
+    }
+  }
+}
 
+// Exact selection over a row in global memory (three radix passes that re-read the row):
+// fills sel[0 .. sortn) with the min(n, topk) selected (key, index) pairs and zero padding.
+// All threads of the block must call it.
+__device__ void select_row_global(const float* __restrict__ x, const int32_t* __restrict__ imap,
+                                  int n, int topk, int sortn, uint64_t* sel, uint32_t* hist,
+                                  uint32_t* warp_sums, uint32_t& s_digit, uint32_t& s_above,
+                                  uint32_t& s_cnt) {
+  const int tid = threadIdx.x;
   if (n <= topk) {
     for (int i = tid; i < sortn; i += kThreads)
       sel[i] = i < n ? compose(score_key(x[i]), imap ? imap[i] : i) : 0ull;
@@ -118,41 +143,443 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(
     for (int i = topk + tid; i < sortn; i += kThreads) sel[i] = 0ull;
   }
   __syncthreads();
+}
 
-  // bitonic sort, descending
-  for (int kk = 2; kk <= sortn; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < (sortn >> 1); i += kThreads) {
-        const int lo = ((i & ~(j - 1)) << 1) | (i & (j - 1));
-        const int hi = lo | j;
-        const uint64_t a = sel[lo], b = sel[hi];
-        const bool desc = (lo & kk) == 0;
-        if (desc ? (a < b) : (a > b)) { sel[lo] = b; sel[hi] = a; }
-      }
+__global__ void __launch_bounds__(kThreads) topk_kernel(
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
+    int sortn, int32_t* __restrict__ idx, float* __restrict__ vals, int64_t row0) {
+  extern __shared__ uint64_t sel[];   // [sortn]
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t s_digit, s_above, s_cnt;
+  const int64_t row = row0 + blockIdx.x;
+  const int n = gather_len ? gather_len[row] : prefix_len(pos, row, L, nullptr);
+  select_row_global(scores + row * stride, index_map ? index_map + row * stride : nullptr, n, topk,
+                    sortn, sel, hist, warp_sums, s_digit, s_above, s_cnt);
+  sort_buf_desc(sel, sortn);
+  write_row(sel, n, topk, row, idx, vals);
+}
+
+// Shared-memory budget of the cluster form (per CTA): the row slice (4 bytes per score)
+// plus the leader's sort buffer (8 bytes per slot); the histogram is static.
+constexpr int kClusterSmemBudget = 200 * 1024;
+constexpr int kSliceTarget = 8192;   // scores per CTA the cluster size aims for
+
+__global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
+    int sortn, int slice_cap, int32_t* __restrict__ idx, float* __restrict__ vals) {
+  extern __shared__ uint8_t dyn[];
+  uint64_t* sel = reinterpret_cast<uint64_t*>(dyn);                     // [sortn] (leader)
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn + (size_t)sortn * 8);  // [slice_cap]
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t s_digit, s_above, s_cnt, s_eq;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int G = (int)cluster.num_blocks();
+  const int crank = (int)cluster.block_rank();
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int64_t row = blockIdx.x / G;
+  const int n = gather_len ? gather_len[row] : prefix_len(pos, row, L, nullptr);
+  const float* x = scores + row * stride;
+  const int32_t* imap = index_map ? index_map + row * stride : nullptr;
+  int slice = (n + G - 1) / G;
+  slice = (slice + 3) & ~3;
+  const int lo = min(n, crank * slice);
+  const int cnt = min(n, lo + slice) - lo;
+  uint64_t* lsel = cluster.map_shared_rank(sel, 0);
+
+  for (int i = tid; i < cnt; i += kThreads) keys[i] = score_key(x[lo + i]);
+  if (tid == 0) { s_cnt = 0; s_eq = 0; }
+  __syncthreads();
+
+  if (n <= topk) {
+    for (int i = tid; i < cnt; i += kThreads)
+      lsel[lo + i] = compose(keys[i], imap ? imap[lo + i] : lo + i);
+    if (crank == 0)
+      for (int i = n + tid; i < sortn; i += kThreads) sel[i] = 0ull;
+    cluster.sync();
+  } else {
+    uint32_t prefix = 0, mask = 0, kneed = (uint32_t)topk;
+    for (int p = 0; p < 3; ++p) {
+      const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+      const int nb = p == 2 ? 1024 : 2048;
+      for (int b = tid; b < kBins; b += kThreads) hist[b] = 0;
       __syncthreads();
+      for (int base = 0; base < cnt; base += kThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < cnt ? keys[i] : 0u;
+        const bool act = i < cnt && (key & mask) == prefix;
+        const uint32_t d = act ? (key >> shift) & (uint32_t)(nb - 1) : 0xffffffffu;
+        // lanes with the same digit add once (scores crowd into few top-level bins)
+        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+        if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
+      }
+      cluster.sync();   // every CTA's histogram is complete
+      const bool on = 2 * tid < nb;
+      uint32_t c_hi = 0, c_lo = 0;
+      if (on) {
+        for (int c = 0; c < G; ++c) {
+          const uint32_t* h = cluster.map_shared_rank(hist, c);
+          c_hi += h[nb - 1 - 2 * tid];
+          c_lo += h[nb - 2 - 2 * tid];
+        }
+      }
+      uint32_t total;
+      const uint32_t excl = block_excl_scan(c_hi + c_lo, warp_sums, total);
+      if (on) {
+        if (excl < kneed && kneed <= excl + c_hi) {
+          s_digit = nb - 1 - 2 * tid;
+          s_above = excl;
+        } else if (excl + c_hi < kneed && kneed <= excl + c_hi + c_lo) {
+          s_digit = nb - 2 - 2 * tid;
+          s_above = excl + c_hi;
+        }
+      }
+      cluster.sync();   // digit known here; no CTA still reads another's histogram
+      prefix |= s_digit << shift;
+      mask |= (uint32_t)(nb - 1) << shift;
+      kneed -= s_above;
     }
+    const uint32_t thr = prefix;
+    // Output slots are fixed without remote atomics: the pairs above the threshold go
+    // first, slice by slice in cluster-rank order; then the equal-to-threshold pairs in
+    // index order, as many as are needed.
+    uint32_t gt_local = 0, eq_local = 0;
+    for (int i = tid; i < cnt; i += kThreads) {
+      gt_local += keys[i] > thr ? 1u : 0u;
+      eq_local += keys[i] == thr ? 1u : 0u;
+    }
+    gt_local = __reduce_add_sync(0xffffffffu, gt_local);
+    eq_local = __reduce_add_sync(0xffffffffu, eq_local);
+    if (lane == 0 && gt_local) atomicAdd(&s_cnt, gt_local);
+    if (lane == 0 && eq_local) atomicAdd(&s_eq, eq_local);
+    cluster.sync();
+    uint32_t gt_base = 0, gt_total = 0, eq_before = 0;
+    for (int c = 0; c < G; ++c) {
+      const uint32_t g = *cluster.map_shared_rank(&s_cnt, c);
+      const uint32_t e = *cluster.map_shared_rank(&s_eq, c);
+      gt_total += g;
+      if (c < crank) { gt_base += g; eq_before += e; }
+    }
+    const uint32_t my_eq = *cluster.map_shared_rank(&s_eq, crank);
+    const uint32_t take_eq = kneed > eq_before ? min(kneed - eq_before, my_eq) : 0u;
+    uint32_t gt_done = 0, eq_done = 0;
+    for (int base = 0; base < cnt; base += kThreads) {
+      const int i = base + tid;
+      const uint32_t key = i < cnt ? keys[i] : 0u;
+      const bool gt = i < cnt && key > thr;
+      const bool eq = i < cnt && key == thr;
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan((gt ? 1u << 16 : 0u) | (eq ? 1u : 0u), warp_sums, tot);
+      if (gt) lsel[gt_base + gt_done + (ex >> 16)] = compose(key, imap ? imap[lo + i] : lo + i);
+      const uint32_t re = eq_done + (ex & 0xffffu);
+      if (eq && re < take_eq)
+        lsel[gt_total + eq_before + re] = compose(key, imap ? imap[lo + i] : lo + i);
+      gt_done += tot >> 16;
+      eq_done += tot & 0xffffu;
+    }
+    if (crank == 0)
+      for (int i = topk + tid; i < sortn; i += kThreads) sel[i] = 0ull;
+    cluster.sync();   // the leader's buffer holds exactly topk pairs
   }
+  if (crank != 0) return;
+  sort_buf_desc(sel, sortn);
+  write_row(sel, n, topk, row, idx, vals);
+}
 
-  const int nvalid = n < topk ? n : topk;
-  for (int i = tid; i < topk; i += kThreads) {
-    const int64_t o = row * topk + i;
-    if (i < nvalid) {
-      const uint64_t v = sel[i];
-      idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
-      if (vals) vals[o] = key_score((uint32_t)(v >> 32));
-    } else {
-      idx[o] = -1;
-      if (vals) vals[o] = __int_as_float(0xff800000);
+// ---------------------------------------------------------------- histogram-split form
+// The score histogram (top kScoreHistBits key bits, one bin = 1/8 octave) gives, for every
+// bin at or above the cutoff bin (the bin of the row's k-th largest score), the output
+// position of its first score.  Those bins are cut into groups by start position
+// (kGroupSpan positions per group); CTA g of a row gathers the scores of group g's bins
+// from the row (a compare-and-compact pass over L2-resident scores), sorts them with a
+// counting sort on the next key bits (groupsort.cuh) and writes them at their positions.
+// Group key ranges are disjoint, so no merge is needed; only the cutoff bin is cut short.
+// Rows whose candidates do not fit (more than kMaxGroups groups, or a bin too large for
+// one group) are done by topk_hist_overflow_kernel with an exact radix select.
+constexpr int kSelThreads = 256;
+constexpr int kGroupSpan = 1024;                          // output positions per group
+constexpr int kMaxGroups = kTopkCandCap / kGroupSpan;     // 16 CTAs per row
+constexpr int kGroupBuf = 4096;                           // pairs one group CTA holds
+constexpr uint32_t kBigBin = kGroupBuf - kGroupSpan;      // larger bins: overflow path
+constexpr int kScatterPer = 16;                           // scores per thread in pass 1
+constexpr int kScatterChunk = kSelThreads * kScatterPer;  // 4096 scores per CTA
+
+// Cutoff bin and candidate statistics of a row from its histogram, identical in every
+// kernel that calls it (NT threads, NT dividing kScoreHistBins).  Thread t owns the
+// bins [hi - kPer, hi), hi = kScoreHistBins - kPer * t; `before` = scores above them.
+template <int NT>
+struct HistView {
+  static constexpr int kPer = kScoreHistBins / NT;
+  uint32_t c[kPer];
+  uint32_t before;
+  int hi;
+};
+
+template <int NT>
+__device__ __forceinline__ uint32_t hist_cutoff(const uint32_t* __restrict__ h, uint32_t target,
+                                                HistView<NT>& v, uint32_t* warp_sums,
+                                                uint32_t& s_cut, uint32_t& s_total,
+                                                uint32_t& s_big) {
+  constexpr int kPer = HistView<NT>::kPer;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  v.hi = kScoreHistBins - kPer * t;
+  uint32_t local = 0;
+  const uint4* h4 = reinterpret_cast<const uint4*>(h + v.hi - kPer);   // 16-byte aligned
+#pragma unroll
+  for (int i = 0; i < kPer / 4; ++i) {
+    const uint4 q = h4[kPer / 4 - 1 - i];
+    v.c[4 * i + 0] = q.w;
+    v.c[4 * i + 1] = q.z;
+    v.c[4 * i + 2] = q.y;
+    v.c[4 * i + 3] = q.x;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) local += v.c[i];
+  if (t == 0) { s_cut = 0; s_total = 0; s_big = 0; }
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t pre = 0;
+  for (int w = 0; w < warp; ++w) pre += warp_sums[w];
+  v.before = pre + incl - local;
+  uint32_t run = v.before;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    if (run < target && target <= run + v.c[i]) s_cut = v.hi - 1 - i;
+    run += v.c[i];
+  }
+  __syncthreads();
+  const uint32_t cut = s_cut;
+  uint32_t cand = 0, big = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    if ((uint32_t)(v.hi - 1 - i) >= cut) {
+      cand += v.c[i];
+      big |= v.c[i] > kBigBin;
+    }
+  if (cand) atomicAdd(&s_total, cand);
+  if (big) s_big = 1;
+  __syncthreads();
+  return cut;
+}
+
+__device__ __forceinline__ bool hist_overflow(uint32_t total, uint32_t big) {
+  return total > (uint32_t)(kMaxGroups * kGroupSpan) || big != 0;
+}
+
+// Output start of every bin at or above the cutoff and the group it belongs to.
+template <int NT>
+__device__ __forceinline__ void bin_groups(const HistView<NT>& hv, uint32_t cut, uint8_t* gid) {
+  uint32_t run = hv.before;
+#pragma unroll
+  for (int i = 0; i < HistView<NT>::kPer; ++i) {
+    const uint32_t b = hv.hi - 1 - i;
+    gid[b] = (b >= cut && hv.c[i]) ? (uint8_t)(run / kGroupSpan) : (uint8_t)0xff;
+    run += hv.c[i];
+  }
+}
+
+// Pass 1: many CTAs per row each read one chunk of the row once and append its
+// candidates (scores in bins at or above the cutoff) to their group's buffer.
+__global__ void __launch_bounds__(kSelThreads) topk_scatter_kernel(
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    const uint32_t* __restrict__ hist, int topk, uint64_t* __restrict__ cand,
+    uint32_t* __restrict__ gcount) {
+  __shared__ uint8_t gid[kScoreHistBins];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t lcount[kMaxGroups], lbase[kMaxGroups];
+  __shared__ uint32_t s_cut, s_total, s_big;
+  const int t = threadIdx.x;
+  const int64_t row = blockIdx.y;
+  const int n = prefix_len(pos, row, L, nullptr);
+  const int start = blockIdx.x * kScatterChunk;
+  if (start >= n) return;
+  if (t < kMaxGroups) lcount[t] = 0;
+  HistView<kSelThreads> hv;
+  const uint32_t cut = hist_cutoff<kSelThreads>(hist + row * kScoreHistBins, (uint32_t)min(n, topk),
+                                                hv, warp_sums, s_cut, s_total, s_big);
+  if (hist_overflow(s_total, s_big)) return;
+  bin_groups<kSelThreads>(hv, cut, gid);
+  const float* x = scores + row * stride;
+  uint32_t key[kScatterPer];
+#pragma unroll
+  for (int j = 0; j < kScatterPer; ++j) {
+    const int e = start + j * kSelThreads + t;
+    key[j] = e < n ? score_key(x[e]) : 0u;
+  }
+  __syncthreads();   // gid complete
+  uint32_t slot[kScatterPer];
+#pragma unroll
+  for (int j = 0; j < kScatterPer; ++j) {
+    const int e = start + j * kSelThreads + t;
+    const uint32_t grp = e < n ? gid[key[j] >> (32 - kScoreHistBits)] : 0xffu;
+    slot[j] = grp != 0xffu ? (grp << 16) | atomicAdd(&lcount[grp], 1u) : 0xffffffffu;
+  }
+  __syncthreads();
+  if (t < kMaxGroups && lcount[t]) lbase[t] = atomicAdd(&gcount[row * kMaxGroups + t], lcount[t]);
+  __syncthreads();
+  uint64_t* crow = cand + row * (int64_t)(kMaxGroups * kGroupBuf);
+#pragma unroll
+  for (int j = 0; j < kScatterPer; ++j) {
+    if (slot[j] == 0xffffffffu) continue;
+    const uint32_t grp = slot[j] >> 16;
+    const uint32_t p = lbase[grp] + (slot[j] & 0xffffu);
+    if (p < (uint32_t)kGroupBuf)
+      crow[grp * kGroupBuf + p] = compose(key[j], start + j * kSelThreads + t);
+  }
+}
+
+// Pass 2: CTA g of a row sorts group g's candidates and writes them at their positions.
+__global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
+    const int32_t* __restrict__ pos, int64_t L, const uint32_t* __restrict__ hist, int topk,
+    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, float* __restrict__ vals) {
+  extern __shared__ uint64_t gbuf[];   // [2 * kGroupBuf]: gathered, then sorted
+  __shared__ uint32_t buckets[kSubBucketWords];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t s_cut, s_total, s_big, s_lo, s_hi, s_start, s_cnt, s_flag;
+  uint64_t* gathered = gbuf;
+  uint64_t* sorted = gbuf + kGroupBuf;
+  const int t = threadIdx.x;
+  const int64_t row = blockIdx.y;
+  const uint32_t g = blockIdx.x;
+  const int n = prefix_len(pos, row, L, nullptr);
+  const uint32_t target = (uint32_t)min(n, topk);
+  if (t == 0) { s_lo = 0xffffffffu; s_hi = 0; s_start = 0xffffffffu; s_cnt = 0; }
+  HistView<kSelThreads> hv;
+  const uint32_t cut = hist_cutoff<kSelThreads>(hist + row * kScoreHistBins, target, hv, warp_sums,
+                                                s_cut, s_total, s_big);
+  if (hist_overflow(s_total, s_big)) return;   // topk_hist_overflow_kernel takes this row
+  {
+    uint32_t run = hv.before, lo = 0xffffffffu, hb = 0, cnt = 0, st = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < HistView<kSelThreads>::kPer; ++i) {
+      const uint32_t b = hv.hi - 1 - i;
+      if (b >= cut && hv.c[i] && run / kGroupSpan == g) {
+        lo = min(lo, b);
+        hb = max(hb, b);
+        cnt += hv.c[i];
+        st = min(st, run);
+      }
+      run += hv.c[i];
+    }
+    if (cnt) {
+      atomicMin(&s_lo, lo);
+      atomicMax(&s_hi, hb);
+      atomicAdd(&s_cnt, cnt);
+      atomicMin(&s_start, st);
     }
   }
+  __syncthreads();
+  if (g == 0)
+    for (int i = target + t; i < topk; i += kSelThreads) {
+      idx[row * topk + i] = -1;
+      if (vals) vals[row * topk + i] = __int_as_float(0xff800000);
+    }
+  const uint32_t cnt = min(s_cnt, (uint32_t)kGroupBuf);
+  if (cnt == 0) return;
+  const uint32_t blo = s_lo, bhi = s_hi, start = s_start;
+  const uint64_t* src = cand + row * (int64_t)(kMaxGroups * kGroupBuf) + g * kGroupBuf;
+  for (uint32_t i = t; i < cnt; i += kSelThreads) gathered[i] = src[i];
+  __syncthreads();
+  if (!group_sort_desc<kSelThreads>(gathered, cnt, sorted, buckets, blo, bhi, warp_sums, s_flag)) {
+    // crowded buckets (many equal scores): bitonic sort of the group instead
+    int sortn = kSelThreads;
+    while ((uint32_t)sortn < cnt) sortn <<= 1;
+    for (int i = t; i < sortn; i += kSelThreads) sorted[i] = (uint32_t)i < cnt ? gathered[i] : 0ull;
+    __syncthreads();
+    switch (sortn / kSelThreads) {   // cnt <= kGroupBuf = 16 * kSelThreads
+      case 1: sort_buf_desc_e<1, kSelThreads>(sorted); break;
+      case 2: sort_buf_desc_e<2, kSelThreads>(sorted); break;
+      case 4: sort_buf_desc_e<4, kSelThreads>(sorted); break;
+      case 8: sort_buf_desc_e<8, kSelThreads>(sorted); break;
+      default: sort_buf_desc_e<16, kSelThreads>(sorted); break;
+    }
+  }
+  for (uint32_t i = t; i < cnt && start + i < target; i += kSelThreads) {
+    const uint64_t v = sorted[i];
+    const int64_t o = row * topk + start + i;
+    idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
+    if (vals) vals[o] = key_score((uint32_t)(v >> 32));
+  }
+}
+
+// Exact selection for the rows topk_group_kernel leaves out (same overflow test).
+__global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    const uint32_t* __restrict__ hist, int topk, int sortn, int32_t* __restrict__ idx,
+    float* __restrict__ vals) {
+  extern __shared__ uint64_t sel[];   // [sortn]
+  __shared__ uint32_t hbuf[kBins];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t s_cut, s_total, s_big, s_digit, s_above, s_cnt;
+  const int64_t row = blockIdx.x;
+  const int n = prefix_len(pos, row, L, nullptr);
+  HistView<kThreads> hv;
+  hist_cutoff<kThreads>(hist + row * kScoreHistBins, (uint32_t)min(n, topk), hv, warp_sums, s_cut,
+                        s_total, s_big);
+  if (!hist_overflow(s_total, s_big)) return;
+  select_row_global(scores + row * stride, nullptr, n, topk, sortn, sel, hbuf, warp_sums, s_digit,
+                    s_above, s_cnt);
+  sort_buf_desc(sel, sortn);
+  write_row(sel, n, topk, row, idx, vals);
 }
 
 }  // namespace
 
 int topk_sort_size(int topk) {
-  int s = 2;
+  int s = kThreads;
   while (s < topk) s <<= 1;
   return s;
+}
+
+cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
+                             const uint32_t* hist, uint64_t* cand, uint32_t* gcount, int rows,
+                             int topk, int32_t* idx, float* vals, cudaStream_t st) {
+  dim3 sgrid((unsigned)((L + kScatterChunk - 1) / kScatterChunk), (unsigned)rows);
+  topk_scatter_kernel<<<sgrid, kSelThreads, 0, st>>>(scores, stride, pos, L, hist, topk, cand,
+                                                     gcount);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)2 * kGroupBuf * sizeof(uint64_t);
+  e = cudaFuncSetAttribute(topk_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_group_kernel<<<dim3(kMaxGroups, (unsigned)rows), kSelThreads, smem, st>>>(
+      pos, L, hist, topk, cand, idx, vals);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int sortn = topk_sort_size(topk);
+  const size_t ov_smem = (size_t)sortn * sizeof(uint64_t);
+  e = cudaFuncSetAttribute(topk_hist_overflow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)ov_smem);
+  if (e != cudaSuccess) return e;
+  topk_hist_overflow_kernel<<<rows, kThreads, ov_smem, st>>>(scores, stride, pos, L, hist, topk,
+                                                             sortn, idx, vals);
+  return cudaGetLastError();
+}
+
+size_t topk_hist_ws_bytes(int64_t rows) {
+  return align256((size_t)rows * kScoreHistBins * 4) + align256((size_t)rows * kMaxGroups * 4) +
+         align256((size_t)rows * kMaxGroups * kGroupBuf * 8);
+}
+
+// Cluster size for rows of up to `len` scores, or 0 when the cluster form does not fit.
+static int cluster_size_for(int64_t len, int sortn) {
+  for (int G = 1; G <= 8; G <<= 1) {
+    const int64_t slice = (((len + G - 1) / G) + 3) & ~int64_t(3);
+    const int64_t smem = (int64_t)sortn * 8 + slice * 4;
+    if ((slice <= kSliceTarget || G == 8) && smem <= kClusterSmemBudget) return G;
+    if (G == 8) break;
+  }
+  return 0;
 }
 
 cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
@@ -160,6 +587,38 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
                         int topk, int32_t* idx, float* vals, int* status, cudaStream_t st) {
   (void)status;
   const int sortn = topk_sort_size(topk);
+  const int64_t maxlen = gather_len ? stride : L;
+  const int G = cluster_size_for(maxlen, sortn);
+  if (G > 0) {
+    const int64_t slice = (((maxlen + G - 1) / G) + 3) & ~int64_t(3);
+    const size_t smem = (size_t)sortn * 8 + (size_t)slice * 4;
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
+      const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(nr * G), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = G;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const int64_t off_rows = row0;
+      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores + off_rows * stride, stride,
+                             pos ? pos + off_rows : nullptr, L,
+                             gather_len ? gather_len + off_rows : nullptr,
+                             index_map ? index_map + off_rows * stride : nullptr, topk, sortn,
+                             (int)slice, idx + off_rows * topk, vals ? vals + off_rows * topk : nullptr);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   const size_t smem = (size_t)sortn * sizeof(uint64_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

@@ -34,14 +34,18 @@ def test_exports_every_declared_symbol(lib):
 
 def test_workspace_sizes(lib):
     ws = lib.misa_workspace_size
-    # route: 256-byte header + rows * chunks * H fp32, chunk = 32 blocks
-    assert ws(1, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 16 * 64 * 4
+    # route: 256-byte header + rows * chunks * H fp32 (chunk = 32 blocks) + row counters
+    assert ws(1, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 16 * 64 * 4 + 256
     # score + top-k: header + rows * L fp32 scores + tensor-core scratch (gathered q rows
     # padded to 16 heads, their weights, per-row tile offsets), each 256-aligned
     a256 = lambda x: (x + 255) // 256 * 256
     tc = lambda rows, n: a256(rows * n * 256) + a256(rows * n * 4) + a256((rows + 1) * 4)
-    assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 16)
-    assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 64)
+    # rows of 8192+ scores (at most 1024 rows) add the histogram top-k scratch: per row a
+    # 4096-bin score histogram, 16 group counts and 16 group buffers of 4096 pairs
+    hp = lambda rows: a256(rows * 4096 * 4) + a256(rows * 16 * 4) + a256(rows * 16 * 4096 * 8)
+    assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 16) + hp(32)
+    assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 64) + hp(32)
+    assert ws(2, 1, 16, 64, 128, 2048, 64, 8, 256, 512) == 256 + 16 * 2048 * 4 + tc(16, 16)
     assert ws(4, 16, 1, 64, 128, 131072, 64, 8, 2048, 8192) == 256 + 2 * 16 * 8192 * 4 + 256
     # invalid sizes report 0
     assert ws(1, 0, 1, 64, 128, 1024, 64, 8, 16, 16) == 0

@@ -70,6 +70,7 @@ extern "C" {
 #define MISA_OP_SCORE_TOPK    2
 #define MISA_OP_DSA_TOPK      3
 #define MISA_OP_DAGGER_RERANK 4
+#define MISA_OP_SCORE_ROWS    5
 
 /* Limits of this build (larger values return MISA_ERR_UNSUPPORTED). */
 #define MISA_HEAD_DIM        128
@@ -130,6 +131,18 @@ int dsa_score_topk(const uint16_t* q, const float* w, const uint16_t* k,
                    const int32_t* pos, int nseq, int T, int H, int d, int64_t L, int topk,
                    int32_t* idx, float* vals, float* scores, void* ws, size_t ws_bytes,
                    void* stream);
+
+/*
+ * Token scores without selection: Eq. (9) over each query's prefix when heads is given
+ * (h heads per query), Eq. (1) with all H heads when heads is NULL.  scores is fp32
+ * [nseq, T, L]; entries s > pos are left untouched.  This is the scoring kernel of
+ * misa_score_topk / dsa_score_topk on its own (same launch configuration), for callers
+ * that select tokens themselves or inspect the scores.
+ * Needs misa_workspace_size(MISA_OP_SCORE_ROWS, ...) (h = H when heads is NULL).
+ */
+int misa_score_rows(const uint16_t* q, const float* w, const uint16_t* k, const int32_t* heads,
+                    const int32_t* pos, int nseq, int T, int H, int d, int64_t L, int h,
+                    float* scores, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * MISA-dagger fine stage, Eq. (12) (Methodology section 2): for each query,

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     misa_dagger_rerank,
     misa_pool_keys,
     misa_route_heads,
+    misa_score_rows,
     misa_score_topk,
     misa_score_topk_noalloc,
     misa_workspace_size,

@@ -41,6 +41,8 @@ _SIGS = {
                                 _p, _p, _p, _p, _c_sz, _p]),
     "misa_dagger_rerank": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_i64,
                                     _c_int, _c_int, _p, _p, _p, _c_sz, _p]),
+    "misa_score_rows": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_i64,
+                                 _c_int, _p, _p, _c_sz, _p]),
     "misa_score_topk_noalloc": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
                                          _c_i64, _c_int, _c_int, _p, _p, _p, _p]),
     "misa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -50,7 +52,7 @@ for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
     _f.restype, _f.argtypes = _res, _args
 
-OP_ROUTE_HEADS, OP_SCORE_TOPK, OP_DSA_TOPK, OP_DAGGER_RERANK = 1, 2, 3, 4
+OP_ROUTE_HEADS, OP_SCORE_TOPK, OP_DSA_TOPK, OP_DAGGER_RERANK, OP_SCORE_ROWS = 1, 2, 3, 4, 5
 HEAD_DIM = 128
 
 
@@ -226,6 +228,31 @@ def dsa_score_topk(q, w, k, pos, topk: int, return_vals: bool = True,
                                _ptr(idx), _ptr(vals), _ptr(scores), _ptr(ws), ws.numel(),
                                _stream()))
     return (idx, vals) if return_vals else idx
+
+
+def misa_score_rows(q, w, k, heads, pos, scores: torch.Tensor | None = None):
+    """Token scores without selection: routed (Eq. 9) when heads is given, dense (Eq. 1)
+    when heads is None.  Returns fp32 [nseq, T, L]; entries past each query's position
+    are left as they were."""
+    q, k = _bits(q, "q"), _bits(k, "k")
+    w = _dev(w, "w", torch.float32)
+    pos = _dev(pos, "pos", torch.int32)
+    nseq, T, H, d = q.shape
+    L = k.shape[1]
+    if heads is not None:
+        heads = _dev(heads, "heads", torch.int32)
+    h = heads.shape[-1] if heads is not None else H
+    if scores is None:
+        scores = torch.empty((nseq, T, L), dtype=torch.float32, device=q.device)
+    _dev(scores, "scores", torch.float32)
+    nb = misa_workspace_size(OP_SCORE_ROWS, nseq, T, H, d, L, 1, h, 1, 1)
+    if nb == 0:
+        raise MisaError("misa_workspace_size", 1)
+    ws = _WS.get(nb, q.device)
+    _check("misa_score_rows",
+           _lib.misa_score_rows(_ptr(q), _ptr(w), _ptr(k), _ptr(heads), _ptr(pos), nseq, T, H, d,
+                                L, h, _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    return scores
 
 
 def misa_dagger_rerank(q, w, k, pos, cand, topk: int, return_vals: bool = True, idx=None,

@@ -90,16 +90,17 @@ size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
 constexpr int kHistPathMaxRows = 1024;
 constexpr int64_t kHistPathMinLen = 8192;
 
-bool hist_path(int nseq, int T, int64_t L) {
-  return (int64_t)nseq * T <= kHistPathMaxRows && L >= kHistPathMinLen;
+bool hist_path(int nseq, int T, int64_t L, int nh) {
+  return (int64_t)nseq * T <= kHistPathMaxRows && L >= kHistPathMinLen &&
+         !score_tc_block_form(nh, T);
 }
 
 size_t hist_path_bytes(int64_t rows) { return topk_hist_ws_bytes(rows); }
 
 size_t score_ws(int nseq, int T, int64_t L, int nh) {
   const int64_t rows = (int64_t)nseq * T;
-  return kStatusBytes + align256((size_t)rows * L * sizeof(float)) + score_tc_ws_bytes(rows, nh) +
-         (hist_path(nseq, T, L) ? hist_path_bytes(rows) : 0);
+  return kStatusBytes + align256((size_t)rows * L * sizeof(float)) +
+         score_tc_ws_bytes(nseq, T, nh) + (hist_path(nseq, T, L, nh) ? hist_path_bytes(rows) : 0);
 }
 size_t dagger_ws(int nseq, int T, int kprime) {
   const size_t rows = (size_t)nseq * T;
@@ -132,6 +133,9 @@ size_t misa_workspace_size(int op, int nseq, int T, int H, int d, int64_t L, int
     case MISA_OP_DSA_TOPK:
       if (check_topk(topk) != MISA_OK) return 0;
       return score_ws(nseq, T, L, H);
+    case MISA_OP_SCORE_ROWS:
+      if (h < 1 || h > H) return 0;
+      return kStatusBytes + score_tc_ws_bytes(nseq, T, h);
     case MISA_OP_DAGGER_RERANK:
       if (check_topk(topk) != MISA_OK || kprime < topk || kprime > MISA_MAX_TOPK) return 0;
       return dagger_ws(nseq, T, kprime);
@@ -194,8 +198,8 @@ static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* 
   if (score_tc_supported(nseq, T, nh, L)) {
     const size_t sc_bytes = align256(rows * L * sizeof(float));
     void* tc_scratch = ws_region(ws, sc_bytes);
-    if (hist_path(nseq, T, L)) {
-      char* hp = ws_region(ws, sc_bytes + score_tc_ws_bytes(rows, nh));
+    if (hist_path(nseq, T, L, nh)) {
+      char* hp = ws_region(ws, sc_bytes + score_tc_ws_bytes(nseq, T, nh));
       const size_t hb = align256(rows * kScoreHistBins * 4);
       const size_t gb = align256(rows * 16 * 4);
       uint32_t* hist = reinterpret_cast<uint32_t*>(hp);
@@ -237,6 +241,30 @@ int dsa_score_topk(const uint16_t* q, const float* w, const uint16_t* k, const i
   MISA_TRY(check_topk(topk));
   return score_topk_common(q, w, k, nullptr, H, pos, nseq, T, H, d, L, topk, idx, vals, scores,
                            ws, ws_bytes, stream);
+}
+
+int misa_score_rows(const uint16_t* q, const float* w, const uint16_t* k, const int32_t* heads,
+                    const int32_t* pos, int nseq, int T, int H, int d, int64_t L, int h,
+                    float* scores, void* ws, size_t ws_bytes, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  if (h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  if (heads && h > MISA_MAX_ROUTED) return MISA_ERR_UNSUPPORTED;
+  const int nh = heads ? h : H;
+  const size_t rows = (size_t)nseq * T;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  if (heads) MISA_TRY(check_dev(heads, rows * h * 4, 4));
+  MISA_TRY(check_dev(scores, rows * L * 4, 4));
+  const size_t need = kStatusBytes + score_tc_ws_bytes(nseq, T, nh);
+  MISA_TRY(check_ws(ws, ws_bytes, need));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (score_tc_supported(nseq, T, nh, L))
+    return cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, scores, L,
+                                       ws_region(ws, 0), status_word(ws), nullptr, st));
+  return cuda_status(launch_score_simt(q, w, k, heads, h, pos, nullptr, nullptr, nseq, T, H, L,
+                                       scores, L, status_word(ws), st));
 }
 
 int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k, const int32_t* pos,

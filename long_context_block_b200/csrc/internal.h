@@ -44,11 +44,13 @@ cudaError_t launch_score_simt(const uint16_t* q, const float* w, const uint16_t*
                               int nseq, int T, int H, int64_t L, float* out,
                               int64_t out_stride, int* status, cudaStream_t st);
 
-// K4 -- token scoring on tcgen05 tensor cores, rows streaming their own key prefix
-// (score_tc.cu).  Same contract as launch_score_simt without the gather mode; needs
-// score_tc_ws_bytes(rows, nh) bytes of 256-aligned scratch.
+// K4 -- token scoring on tcgen05 tensor cores (score_tc.cu): rows streaming their own key
+// prefix (decode form), or blocks of queries sharing key tiles (block form, when a
+// sequence has enough queries).  Same contract as launch_score_simt without the gather
+// mode; needs score_tc_ws_bytes(nseq, T, nh) bytes of 256-aligned scratch.
 bool score_tc_supported(int nseq, int T, int nh, int64_t L);
-size_t score_tc_ws_bytes(int64_t rows, int nh);
+bool score_tc_block_form(int nh, int T);
+size_t score_tc_ws_bytes(int nseq, int T, int nh);
 //   hist (nullable, zeroed by the caller): per-row kScoreHistBins-bin histogram of the
 //   written scores' keys, accumulated in the epilogue.
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,

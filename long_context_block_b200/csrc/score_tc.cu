@@ -1,25 +1,30 @@
-// K4 (tensor-core form): indexer token scores on tcgen05 for rows that each stream their
-// own prefix of keys (decode: one query per sequence).
+// K4 (tensor-core form): indexer token scores on tcgen05.
 //
 //   routed (Eq. 9):  Ihat[t,s] = sum_{r < h} w[t,H_t[r]] * ReLU(q[t,H_t[r]] . k[s])
 //   dense  (Eq. 1):  I[t,s]    = sum_{j < H} w[t,j]      * ReLU(q[t,j] . k[s])
 //
-// Per 128-key tile the contraction S[s, r] = k[s] . q_r is one tcgen05 MMA chain
-// (M = 128 keys, N = the row's head count padded to a multiple of 16, K = 128 in
-// eight K = 16 steps) with both operands in shared memory and the fp32 result in TMEM.
-// The operation is HBM-bound (256 bytes of keys per token against 2*N*128 flops), so
-// the kernel is built around the key stream:
+// Work unit: QB consecutive query rows of one sequence, each with HS head slots (the
+// routed heads, or all heads, zero-padded).  Their q vectors form the MMA's B operand
+// (N = QB * HS rows of 128 bf16, resident in shared memory for the unit), and the
+// unit's causal prefix of keys streams through as the A operand in 128-key tiles
+// (M = 128), K = 128 in eight K = 16 steps, fp32 accumulators in TMEM:
+//   S[s, q*HS + r] = k[s] . q_{t0+q, slot r}.
+// The epilogue applies ReLU, the slot weights and the sum over a query's slots, so each
+// (query, key) score leaves the SM once, as fp32.
+//   * decode form (QB = 1): every row streams its own prefix; the contraction is
+//     HBM-bound (256 bytes of keys per token), N = HS <= 128.
+//   * block form (QB = 256 / HS): QB queries share every key tile, N = 256; the
+//     contraction is tensor-bound (prefill), 2 * 128 * 256 * 128 flops per tile.
 //
-//   warp 0     TMA producer: a ring of kStages 32 KB key tiles (two 64-column boxes,
-//              128-byte swizzle) plus a double-buffered tile of the row's gathered q;
-//   warp 1     MMA issuer (one thread) and TMEM owner;
-//   warps 2-5  epilogue: tcgen05.ld of the thread's key row (TMEM lane), then the fused
-//              ReLU, w-weighting and head sum, and one coalesced fp32 store per key.
-//
-// The grid is persistent (one CTA per SM); the rows' key tiles are laid end to end and
-// every CTA takes a contiguous range of them, so long and short rows balance.  Every
-// wait is bounded: on expiry the kernel records MISA_ERR_DEVICE_TIMEOUT, lets its
-// in-flight copies and MMAs finish, frees TMEM and returns.
+// Warp roles: warp 0 TMA producer (ring of 32 KB key tiles, each two 64-column boxes with
+// the 128-byte swizzle; per unit the q tile and its weights); warp 1 MMA issuer (one
+// thread) and TMEM owner; the epilogue warps (4 in decode form, 8 in block form) read
+// their TMEM lane quarter with tcgen05.ld.  The grid is persistent (one CTA per SM); the
+// units' key tiles are laid end to end and every CTA takes a contiguous range of them,
+// so long and short units balance.  Every wait is bounded: on expiry the kernel records
+// MISA_ERR_DEVICE_TIMEOUT, lets its in-flight copies and MMAs finish, frees TMEM and
+// returns.  In decode form the epilogue can also build a per-row histogram of the score
+// keys for the top-k that follows.
 #include <cuda.h>
 
 #include <mutex>
@@ -35,38 +40,52 @@ using namespace sm100;
 constexpr int kTileKeys = 128;
 constexpr int kKeyTileBytes = kTileKeys * kHeadDim * 2;   // 32 KB
 constexpr int kKeyHalfBytes = kKeyTileBytes / 2;           // [128 rows][64 cols] bf16
-constexpr int kThreads = 192;
 constexpr long long kWaitCycles = 4000000000LL;            // ~2 s at the top SM clock
+constexpr int kSmemLimit = 227 * 1024;
 
-template <int N>
-struct DecodeCfg {
-  static constexpr int kStages = N <= 16 ? 6 : (N <= 64 ? 5 : 4);
+template <int HS, int QB>
+struct Cfg {
+  static constexpr int N = HS * QB;
+  static constexpr int kEpiWarps = QB == 1 ? 4 : 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kAcc = N <= 32 ? 8 : (N <= 64 ? 4 : 2);
-  // accumulator buffers start on power-of-two column offsets
-  static constexpr int kAccStride = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : 128;
-  static constexpr int kCols = (kAcc * kAccStride) <= 32 ? 32 : (kAcc * kAccStride) <= 64 ? 64
-                               : (kAcc * kAccStride) <= 128 ? 128 : 256;
+  static constexpr int kAccStride = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  static constexpr int kCols = kAcc * kAccStride <= 32 ? 32 : kAcc * kAccStride <= 64 ? 64
+                               : kAcc * kAccStride <= 128 ? 128 : kAcc * kAccStride <= 256 ? 256 : 512;
   static constexpr int kQBytes = N * kHeadDim * 2;
   static constexpr int kQHalf = kQBytes / 2;
+  static constexpr int kWBytes = N * 4;
+  // units are short in decode form (double-buffer the q tile), long in block form; the
+  // slot weights are always double-buffered (the epilogue reads them after the MMAs)
+  static constexpr int kQBufs = QB == 1 ? 2 : 1;
+  static constexpr int kWBufs = 2;
+  static constexpr int kHistBytes = QB == 1 ? kScoreHistBins * 4 : 0;
+  static constexpr int kFixed = kQBufs * kQBytes + kWBufs * kWBytes + kHistBytes +
+                                1024 /*bars, misc*/ + 1024 /*alignment*/;
+  static constexpr int kStages0 = (kSmemLimit - kFixed) / kKeyTileBytes;
+  static constexpr int kStages = kStages0 > 6 ? 6 : kStages0;
   static constexpr int kStageBase = 0;
   static constexpr int kQBase = kStages * kKeyTileBytes;
-  static constexpr int kBarBase = kQBase + 2 * kQBytes;
-  // full[S], empty[S], qfull[2], qempty[2], accfull[A], accempty[A], drain
-  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
+  static constexpr int kWBase = kQBase + kQBufs * kQBytes;
+  static constexpr int kHistBase = kWBase + kWBufs * kWBytes;
+  static constexpr int kBarBase = kHistBase + kHistBytes;
+  // full[S], empty[S], qfull[2], qempty[2], wfull[2], wempty[2], accfull[A], accempty[A], drain
+  static constexpr int kNumBars = 2 * kStages + 8 + 2 * kAcc + 1;
   static constexpr int kMiscBase = kBarBase + kNumBars * 8;
-  static constexpr int kHistBase = kMiscBase + 16;            // [kScoreHistBins] u32
-  static constexpr int kSmemBytes = kHistBase + kScoreHistBins * 4 + 1024;   // + alignment slack
-  static_assert(N % 16 == 0 && N >= 16 && N <= 128, "N");
+  static constexpr int kSmemBytes = kMiscBase + 16 + 1024;
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N");
   static_assert(kQHalf % 1024 == 0, "q half tile must keep the 1 KB swizzle alignment");
+  static_assert(kStages >= 3, "key ring too shallow");
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
 
-// Row segment of a CTA's tile range: row r contributes its local tiles [a, b).
+// Unit segment of a CTA's tile range: unit u contributes its local tiles [a, b).
 struct Seg {
-  int r, a, b;
+  int u, a, b;
 };
 
-__device__ __forceinline__ int find_row(const int32_t* off, int rows, int t) {
-  int lo = 0, hi = rows - 1;   // largest r with off[r] <= t
+__device__ __forceinline__ int find_unit(const int32_t* off, int units, int t) {
+  int lo = 0, hi = units - 1;   // largest u with off[u] <= t
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (off[mid] <= t) lo = mid; else hi = mid - 1;
@@ -74,15 +93,15 @@ __device__ __forceinline__ int find_row(const int32_t* off, int rows, int t) {
   return lo;
 }
 
-__device__ __forceinline__ bool next_seg(const int32_t* off, int rows, int t0, int t1, int& r,
+__device__ __forceinline__ bool next_seg(const int32_t* off, int units, int t0, int t1, int& u,
                                          Seg& s) {
-  if (r >= rows) return false;
-  const int o0 = off[r], o1 = off[r + 1];
+  if (u >= units) return false;
+  const int o0 = off[u], o1 = off[u + 1];
   if (o0 >= t1) return false;
-  s.r = r;
+  s.u = u;
   s.a = max(t0, o0) - o0;
   s.b = min(t1, o1) - o0;
-  ++r;
+  ++u;
   return true;
 }
 
@@ -100,17 +119,31 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   mbar_wait(bar, parity, &never, status, kWaitCycles);
 }
 
-template <int N>
-__global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
+__device__ __forceinline__ void epi_bar(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Geometry of the units: sequence n holds ublk = ceil(T / QB) units; unit u covers rows
+// t = (u % ublk) * QB + q, q < QB, t < T.
+struct Units {
+  int T, QB, ublk;
+  __device__ __forceinline__ int seq(int u) const { return u / ublk; }
+  __device__ __forceinline__ int t0(int u) const { return (u % ublk) * QB; }
+};
+
+template <int HS, int QB>
+__global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ wsel, const int32_t* __restrict__ pos,
-    const int32_t* __restrict__ tile_off, int rows, int T, int64_t L, float* __restrict__ out,
-    int64_t out_stride, int* status, uint32_t* __restrict__ hist) {
-  using C = DecodeCfg<N>;
+    const int32_t* __restrict__ tile_off, int units, Units geo, int64_t L,
+    float* __restrict__ out, int64_t out_stride, int* status, uint32_t* __restrict__ hist) {
+  using C = Cfg<HS, QB>;
+  constexpr int N = C::N;
+  constexpr int kEpiThreads = 32 * C::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  const int total = tile_off[rows];
+  const int total = tile_off[units];
   const int t0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
   const int t1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   if (t0 >= t1) return;
@@ -122,19 +155,28 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
   uint64_t* empty = full + C::kStages;
   uint64_t* qfull = empty + C::kStages;
   uint64_t* qempty = qfull + 2;
-  uint64_t* accfull = qempty + 2;
+  uint64_t* wfull = qempty + 2;
+  uint64_t* wempty = wfull + 2;
+  uint64_t* accfull = wempty + 2;
   uint64_t* accempty = accfull + C::kAcc;
   uint64_t* drain = accempty + C::kAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::kMiscBase);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + C::kMiscBase + 4);
   uint32_t* shist = reinterpret_cast<uint32_t*>(base + C::kHistBase);
-  if (hist)
-    for (int b = tid; b < kScoreHistBins; b += kThreads) shist[b] = 0;
+  if (QB == 1 && hist)
+    for (int b = tid; b < kScoreHistBins; b += C::kThreads) shist[b] = 0;
 
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
-    for (int a = 0; a < C::kAcc; ++a) { mbar_init(&accfull[a], 1); mbar_init(&accempty[a], 128); }
+    for (int s = 0; s < C::kQBufs; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
+    for (int s = 0; s < C::kWBufs; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], C::kEpiWarps);   // one arrival per epilogue warp
+    }
+    for (int a = 0; a < C::kAcc; ++a) {
+      mbar_init(&accfull[a], 1);
+      mbar_init(&accempty[a], kEpiThreads);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -144,27 +186,38 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int r_first = find_row(tile_off, rows, t0);
+  const int u_first = find_unit(tile_off, units, t0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    int issued = 0, qissued = 0;
+    int issued = 0, qissued = 0, wissued = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_q);
-      int r = r_first;
+      int u = u_first;
       Seg sg;
       bool ok = true;
-      while (ok && next_seg(tile_off, rows, t0, t1, r, sg)) {
-        const int slot = qissued & 1;
-        if (!mbar_wait(&qempty[slot], ((qissued >> 1) & 1) ^ 1, abort_flag, status, kWaitCycles))
+      while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
+        const int slot = qissued % C::kQBufs;
+        if (!mbar_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status,
+                       kWaitCycles))
           break;
         uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
         mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
-        tma_load_2d(qb, &tm_q, &qfull[slot], 0, sg.r * N);
-        tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.r * N);
+        tma_load_2d(qb, &tm_q, &qfull[slot], 0, sg.u * N);
+        tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
+        const int wslot = qissued % C::kWBufs;
+        if (!mbar_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status,
+                       kWaitCycles)) {
+          ++qissued;
+          break;
+        }
+        mbar_arrive_expect_tx(&wfull[wslot], C::kWBytes);
+        bulk_load(base + C::kWBase + wslot * C::kWBytes, wsel + (int64_t)sg.u * N, C::kWBytes,
+                  &wfull[wslot]);
         ++qissued;
-        const int64_t y0 = (int64_t)(sg.r / T) * L;
+        ++wissued;
+        const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
         for (int j = sg.a; j < sg.b; ++j) {
           const int s = issued % C::kStages;
           if (!mbar_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status,
@@ -185,7 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
     if (lane == 0) {   // let this CTA's own copies land before the CTA exits
       for (int i = max(0, issued - C::kStages); i < issued; ++i)
         drain_wait(&full[i % C::kStages], (i / C::kStages) & 1, status);
-      for (int i = max(0, qissued - 2); i < qissued; ++i) drain_wait(&qfull[i & 1], (i >> 1) & 1, status);
+      for (int i = max(0, qissued - C::kQBufs); i < qissued; ++i)
+        drain_wait(&qfull[i % C::kQBufs], (i / C::kQBufs) & 1, status);
+      for (int i = max(0, wissued - C::kWBufs); i < wissued; ++i)
+        drain_wait(&wfull[i % C::kWBufs], (i / C::kWBufs) & 1, status);
     }
     __syncthreads();   // (B)
   } else if (warp == 1) {
@@ -194,12 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
       constexpr uint32_t idesc = idesc_bf16_f32(128, N);
       const uint32_t smem0 = smem_u32(base);
       int it = 0, acc_it = 0, seg = 0;
-      int r = r_first;
+      int u = u_first;
       Seg sg;
       bool ok = true;
-      while (ok && next_seg(tile_off, rows, t0, t1, r, sg)) {
-        const int slot = seg & 1;
-        if (!mbar_wait(&qfull[slot], (seg >> 1) & 1, abort_flag, status, kWaitCycles)) break;
+      while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
+        const int slot = seg % C::kQBufs;
+        if (!mbar_wait(&qfull[slot], (seg / C::kQBufs) & 1, abort_flag, status, kWaitCycles)) break;
         const uint32_t qaddr = smem0 + C::kQBase + slot * C::kQBytes;
         for (int j = sg.a; j < sg.b; ++j) {
           const int s = it % C::kStages;
@@ -237,77 +293,111 @@ __global__ void __launch_bounds__(kThreads, 1) score_tc_decode_kernel(
     tmem_dealloc(tmem_base, C::kCols);
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;   // TMEM lanes this warp may read
+    constexpr int kColsPerWarp = N / (C::kEpiWarps / 4);   // column share of a warp
+    constexpr int kQPerWarp = QB == 1 ? 1 : kColsPerWarp / HS;
+    const int e = warp - 2;
+    const int quarter = warp & 3;                 // TMEM lanes this warp may read
+    const int col0 = (e / 4) * kColsPerWarp;      // first accumulator column of this warp
+    const int q0 = QB == 1 ? 0 : col0 / HS;       // first query of this warp in the unit
     const int key_in_tile = quarter * 32 + lane;
-    const int etid = tid - 64;      // 0..127 over the four epilogue warps
-    int acc_it = 0;
-    int r = r_first;
+    const int etid = tid - 64;
+    // Every epilogue warp walks the same segments and tiles whatever happens, so the
+    // named barriers of the histogram flush always match; after a failed (bounded) wait a
+    // warp only skips the work.
+    int acc_it = 0, seg = 0;
+    int u = u_first;
     Seg sg;
     bool ok = true;
-    while (ok && next_seg(tile_off, rows, t0, t1, r, sg)) {
-      const int P = prefix_len(pos, sg.r, L, nullptr);
-      float wv[N];
+    while (next_seg(tile_off, units, t0, t1, u, sg)) {
+      const int n = geo.seq(sg.u);
+      const int tq0 = geo.t0(sg.u);
+      int P[kQPerWarp];   // prefix length of each of this warp's queries (0: no query)
 #pragma unroll
-      for (int c = 0; c < N; ++c) wv[c] = __ldg(wsel + (int64_t)sg.r * N + c);
-      float* orow = out + (int64_t)sg.r * out_stride;
-      for (int j = sg.a; j < sg.b; ++j) {
+      for (int q = 0; q < kQPerWarp; ++q) {
+        const int t = tq0 + q0 + q;
+        P[q] = t < geo.T ? prefix_len(pos, (int64_t)n * geo.T + t, L, nullptr) : 0;
+      }
+      // this warp's queries are consecutive rows of the output
+      float* obase = out + ((int64_t)n * geo.T + min(tq0 + q0, geo.T - 1)) * out_stride;
+      const int wslot = seg % C::kWBufs;
+      if (ok && !warp_wait(&wfull[wslot], (seg / C::kWBufs) & 1, abort_flag, status)) ok = false;
+      const float* wsm = reinterpret_cast<const float*>(base + C::kWBase + wslot * C::kWBytes);
+      for (int j = sg.a; j < sg.b && ok; ++j) {
         const int acc = acc_it % C::kAcc;
         if (!warp_wait(&accfull[acc], (acc_it / C::kAcc) & 1, abort_flag, status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t taddr =
-            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::kAccStride);
-        float sc = 0.f;
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                               (uint32_t)(acc * C::kAccStride + col0);
+        float sc[kQPerWarp];
 #pragma unroll
-        for (int c0 = 0; c0 < N; c0 += 16) {
+        for (int q = 0; q < kQPerWarp; ++q) sc[q] = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < kColsPerWarp; c0 += 16) {
           float v[16];
           tmem_ld16(taddr + c0, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) sc = fmaf(wv[c0 + i], fmaxf(v[i], 0.f), sc);
+          for (int i = 0; i < 16; ++i) {
+            const int col = c0 + i;
+            const int q = QB == 1 ? 0 : col / HS;
+            sc[q] = fmaf(wsm[col0 + col], fmaxf(v[i], 0.f), sc[q]);
+          }
         }
         tc_fence_before();
         mbar_arrive(&accempty[acc]);
         const int s = j * kTileKeys + key_in_tile;
-        if (s < P) {
-          orow[s] = sc;
-          if (hist) atomicAdd(&shist[score_key(sc) >> (32 - kScoreHistBits)], 1u);
+#pragma unroll
+        for (int q = 0; q < kQPerWarp; ++q) {
+          if (s < P[q]) {
+            obase[(int64_t)q * out_stride + s] = sc[q];
+            if (QB == 1 && hist) atomicAdd(&shist[score_key(sc[q]) >> (32 - kScoreHistBits)], 1u);
+          }
         }
         ++acc_it;
       }
-      if (hist) {
-        // flush this row's histogram; the four epilogue warps are always in the same
-        // segment here, and leave together (the abort flag is read after the barrier)
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        uint32_t* gh = hist + (int64_t)sg.r * kScoreHistBins;
-        for (int b = etid; b < kScoreHistBins; b += 128) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[wslot]);   // this warp is done with the weights
+      if (QB == 1 && hist) {
+        // flush this row's histogram (all epilogue warps are in this segment)
+        epi_bar(kEpiThreads);
+        uint32_t* gh = hist + (int64_t)sg.u * kScoreHistBins;
+        for (int b = etid; b < kScoreHistBins; b += kEpiThreads) {
           const uint32_t v = shist[b];
-          if (v) { atomicAdd(gh + b, v); shist[b] = 0; }
+          if (v) {
+            if (ok) atomicAdd(gh + b, v);
+            shist[b] = 0;
+          }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        ok = *abort_flag == 0;
+        epi_bar(kEpiThreads);
       }
+      ++seg;
     }
     __syncthreads();   // (A)
     __syncthreads();   // (B)
   }
 }
 
-// Gather the row's head vectors (routed heads, or all heads) into a zero-padded
-// [rows, N, 128] bf16 operand and their weights into [rows, N]; block 0 also lays the
-// rows' key tiles end to end (tile_off[r] = tiles of rows < r).
+// Gather each unit's head vectors (routed heads, or all heads) into a zero-padded
+// [units, QB * HS, 128] bf16 operand and their weights into [units, QB * HS]; block 0
+// also lays the units' key tiles end to end (tile_off[u] = tiles of units < u).
 __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
     const uint16_t* __restrict__ q, const float* __restrict__ w, const int32_t* __restrict__ heads,
-    int hsel, int H, int N, const int32_t* __restrict__ pos, int rows, int64_t L,
+    int hsel, int H, int HS, Units geo, const int32_t* __restrict__ pos, int units, int64_t L,
     uint4* __restrict__ qg, float* __restrict__ wg, int32_t* __restrict__ tile_off, int* status) {
-  const int64_t row = blockIdx.x;
+  const int u = blockIdx.x;
   const int tid = threadIdx.x;
   const int nh = heads ? hsel : H;
+  const int N = HS * geo.QB;
+  const int n = geo.seq(u), tq0 = geo.t0(u);
   for (int e = tid; e < N * 16; e += blockDim.x) {
-    const int r = e >> 4, c = e & 15;
+    const int col = e >> 4, c = e & 15;
+    const int qq = col / HS, r = col % HS;
+    const int t = tq0 + qq;
+    const int64_t row = (int64_t)n * geo.T + t;
     int j = -1;
-    if (r < nh) {
+    if (t < geo.T && r < nh) {
       j = heads ? heads[row * hsel + r] : r;
       if (j < 0 || j >= H) {
         if (c == 0) set_status(status, MISA_ERR_BAD_DEVICE_INPUT);
@@ -316,20 +406,23 @@ __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
     }
     uint4 v = make_uint4(0, 0, 0, 0);
     if (j >= 0) v = reinterpret_cast<const uint4*>(q + (row * H + j) * kHeadDim)[c];
-    qg[(row * N + r) * 16 + c] = v;
-    if (c == 0) wg[row * N + r] = j >= 0 ? w[row * H + j] : 0.f;
+    qg[((int64_t)u * N + col) * 16 + c] = v;
+    if (c == 0) wg[(int64_t)u * N + col] = j >= 0 ? w[row * H + j] : 0.f;
   }
   if (blockIdx.x == 0) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     if (tid == 0) carry = 0;
     __syncthreads();
-    for (int base = 0; base < rows; base += blockDim.x) {
-      const int rr = base + tid;
+    for (int base = 0; base < units; base += blockDim.x) {
+      const int uu = base + tid;
       int v = 0;
-      if (rr < rows) {
-        const int P = prefix_len(pos, rr, L, status);
-        v = (P + kTileKeys - 1) / kTileKeys;
+      if (uu < units) {
+        const int nn = geo.seq(uu), ta = geo.t0(uu);
+        int Pmax = 0;
+        for (int qq = 0; qq < geo.QB && ta + qq < geo.T; ++qq)
+          Pmax = max(Pmax, prefix_len(pos, (int64_t)nn * geo.T + ta + qq, L, status));
+        v = (Pmax + kTileKeys - 1) / kTileKeys;
       }
       int incl = v;
 #pragma unroll
@@ -350,12 +443,12 @@ __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
       }
       __syncthreads();
       const int excl = carry + (tid >= 32 ? warp_tot[(tid >> 5) - 1] : 0) + incl - v;
-      if (rr < rows) tile_off[rr] = excl;
+      if (uu < units) tile_off[uu] = excl;
       __syncthreads();
       if (tid == blockDim.x - 1) carry = excl + v;
       __syncthreads();
     }
-    if (tid == 0) tile_off[rows] = carry;
+    if (tid == 0) tile_off[units] = carry;
   }
 }
 
@@ -393,73 +486,109 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t nrows, uint32_t box_rows
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N>
-cudaError_t launch_n(const CUtensorMap& tk, const CUtensorMap& tq, const float* wg,
-                     const int32_t* pos, const int32_t* tile_off, int rows, int T, int64_t L,
-                     float* out, int64_t out_stride, int* status, uint32_t* hist,
-                     cudaStream_t st) {
-  using C = DecodeCfg<N>;
-  cudaError_t e = cudaFuncSetAttribute(score_tc_decode_kernel<N>,
+template <int HS, int QB>
+cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float* wg,
+                       const int32_t* pos, const int32_t* tile_off, int units, Units geo,
+                       int64_t L, float* out, int64_t out_stride, int* status, uint32_t* hist,
+                       cudaStream_t st) {
+  using C = Cfg<HS, QB>;
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  score_tc_decode_kernel<N><<<sms, kThreads, C::kSmemBytes, st>>>(
-      tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist);
+  score_tc_kernel<HS, QB><<<sms, C::kThreads, C::kSmemBytes, st>>>(
+      tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist);
   return cudaGetLastError();
+}
+
+// Shape of the work units for nh heads and T queries per sequence.
+struct Plan {
+  int HS, QB, N;
+};
+
+Plan plan_for(int nh, int T) {
+  Plan p;
+  // block form when a sequence has enough queries to fill a 256-column B operand
+  const int hs_pow2 = nh <= 8 ? 8 : nh <= 16 ? 16 : nh <= 32 ? 32 : nh <= 64 ? 64 : 128;
+  const int qb = 256 / hs_pow2;
+  if (T >= qb && T >= 16) {
+    p.HS = hs_pow2;
+    p.QB = qb;
+  } else {
+    p.HS = ((nh + 15) / 16) * 16;
+    p.QB = 1;
+  }
+  p.N = p.HS * p.QB;
+  return p;
 }
 
 }  // namespace
 
-int score_tc_padded_heads(int nh) { return ((nh + 15) / 16) * 16; }
-
-size_t score_tc_ws_bytes(int64_t rows, int nh) {
-  const int64_t N = score_tc_padded_heads(nh);
-  return align256((size_t)rows * N * kHeadDim * 2) + align256((size_t)rows * N * 4) +
-         align256((size_t)(rows + 1) * 4);
+size_t score_tc_ws_bytes(int nseq, int T, int nh) {
+  const Plan p = plan_for(nh, T);
+  const int64_t units = (int64_t)nseq * ((T + p.QB - 1) / p.QB);
+  return align256((size_t)units * p.N * kHeadDim * 2) + align256((size_t)units * p.N * 4) +
+         align256((size_t)(units + 1) * 4);
 }
 
+bool score_tc_block_form(int nh, int T) { return plan_for(nh, T).QB > 1; }
+
 bool score_tc_supported(int nseq, int T, int nh, int64_t L) {
-  const int64_t rows = (int64_t)nseq * T;
-  const int64_t tiles = rows * ((L + kTileKeys - 1) / kTileKeys);
+  const Plan p = plan_for(nh, T);
+  const int64_t units = (int64_t)nseq * ((T + p.QB - 1) / p.QB);
+  const int64_t tiles = units * ((L + kTileKeys - 1) / kTileKeys);
   return nh >= 1 && nh <= 128 && (int64_t)nseq * L < INT32_MAX && tiles < INT32_MAX &&
-         rows * score_tc_padded_heads(nh) < INT32_MAX && encode_fn() != nullptr;
+         units * p.N < INT32_MAX && encode_fn() != nullptr;
 }
 
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
                             int* status, uint32_t* hist, cudaStream_t st) {
-  const int rows = nseq * T;
   const int nh = heads ? hsel : H;
-  const int N = score_tc_padded_heads(nh);
-  char* p = reinterpret_cast<char*>(scratch);
-  uint4* qg = reinterpret_cast<uint4*>(p);
-  p += align256((size_t)rows * N * kHeadDim * 2);
-  float* wg = reinterpret_cast<float*>(p);
-  p += align256((size_t)rows * N * 4);
-  int32_t* tile_off = reinterpret_cast<int32_t*>(p);
+  const Plan p = plan_for(nh, T);
+  Units geo;
+  geo.T = T;
+  geo.QB = p.QB;
+  geo.ublk = (T + p.QB - 1) / p.QB;
+  const int units = nseq * geo.ublk;
+  char* c = reinterpret_cast<char*>(scratch);
+  uint4* qg = reinterpret_cast<uint4*>(c);
+  c += align256((size_t)units * p.N * kHeadDim * 2);
+  float* wg = reinterpret_cast<float*>(c);
+  c += align256((size_t)units * p.N * 4);
+  int32_t* tile_off = reinterpret_cast<int32_t*>(c);
+  if (p.QB > 1) hist = nullptr;
 
-  score_tc_prep_kernel<<<rows, 1024, 0, st>>>(q, w, heads, hsel, H, N, pos, rows, L, qg, wg,
-                                              tile_off, status);
+  score_tc_prep_kernel<<<units, 1024, 0, st>>>(q, w, heads, hsel, H, p.HS, geo, pos, units, L, qg,
+                                               wg, tile_off, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tk, tq;
   if (!make_map(&tk, k, (uint64_t)nseq * L, kTileKeys) ||
-      !make_map(&tq, qg, (uint64_t)rows * N, (uint32_t)N))
+      !make_map(&tq, qg, (uint64_t)units * p.N, (uint32_t)p.N))
     return cudaErrorInvalidValue;
-  switch (N) {
-    case 16: return launch_n<16>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 32: return launch_n<32>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 48: return launch_n<48>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 64: return launch_n<64>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 80: return launch_n<80>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 96: return launch_n<96>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 112: return launch_n<112>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    case 128: return launch_n<128>(tk, tq, wg, pos, tile_off, rows, T, L, out, out_stride, status, hist, st);
-    default: return cudaErrorInvalidValue;
-  }
+#define MISA_TC_CASE(HS_, QB_)                                                                  \
+  if (p.HS == HS_ && p.QB == QB_)                                                               \
+    return launch_cfg<HS_, QB_>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, \
+                                hist, st);
+  MISA_TC_CASE(16, 1)
+  MISA_TC_CASE(32, 1)
+  MISA_TC_CASE(48, 1)
+  MISA_TC_CASE(64, 1)
+  MISA_TC_CASE(80, 1)
+  MISA_TC_CASE(96, 1)
+  MISA_TC_CASE(112, 1)
+  MISA_TC_CASE(128, 1)
+  MISA_TC_CASE(8, 32)
+  MISA_TC_CASE(16, 16)
+  MISA_TC_CASE(32, 8)
+  MISA_TC_CASE(64, 4)
+  MISA_TC_CASE(128, 2)
+#undef MISA_TC_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace misa

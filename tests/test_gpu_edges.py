@@ -130,3 +130,29 @@ def test_guard_bands_untouched(M):
     torch.cuda.synchronize()
     for buf, fill in ((kp_buf, 7.0), (h_buf, 77), (e_buf, 7.0), (i_buf, 77), (v_buf, 7.0)):
         assert torch.all(buf[:G] == fill) and torch.all(buf[-G:] == fill)
+
+
+@pytest.mark.parametrize("T,pos_mode", [(3, "tail"), (70, "causal")])
+def test_score_rows_entry_point(M, T, pos_mode):
+    """misa_score_rows (scores without selection) against the oracle's Eq. (9) under the
+    GPU's heads and Eq. (1), for decode-form rows and for query blocks (T >= 32)."""
+    import oracle.misa_oracle as orc
+    from tests import tolerance as tl
+    wl = _wl(nseq=2, T=T, L=900, topk=32, kprime=64, pos_mode=pos_mode)
+    x = make_inputs(wl, seed=13)
+    q, w, k, pos = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, wl.B)
+    heads = M.misa_route_heads(q, w, k, kp, pos, wl.B, wl.h)
+    routed = M.misa_score_rows(q, w, k, heads, pos).cpu().numpy()
+    dense = M.misa_score_rows(q, w, k, None, pos).cpu().numpy()
+    hh = heads.cpu().numpy()
+    for n in range(wl.nseq):
+        kk = orc.bf16_bits_to_f64(x.k_bits[n])
+        for t in range(T):
+            P = int(x.pos[n, t]) + 1
+            q_t = orc.bf16_bits_to_f64(x.q_bits[n, t])
+            w_t = x.w[n, t].astype(np.float64)
+            tl.check_scores(routed[n, t, :P], orc.token_scores(q_t, w_t, kk, P, hh[n, t]),
+                            what=f"routed {n},{t}")
+            tl.check_scores(dense[n, t, :P], orc.dense_scores(q_t, w_t, kk, P),
+                            what=f"dense {n},{t}")

@@ -80,6 +80,7 @@ int check_topk(int topk) {
 }
 
 size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
+  if (route_tc_supported(nseq, T, H, L, B)) return kStatusBytes + route_tc_ws_bytes(nseq, T, H);
   const int64_t M = (L + B - 1) / B;
   const int64_t nchunk = (M + kRouteChunk - 1) / kRouteChunk;
   return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float)) +
@@ -169,6 +170,9 @@ int misa_route_heads(const uint16_t* q, const float* w, const uint16_t* k, const
   MISA_TRY(check_dev(heads, rows * h * 4, 4));
   MISA_TRY(check_opt(E, rows * H * 4, 4));
   MISA_TRY(check_ws(ws, ws_bytes, route_ws(nseq, T, H, L, B)));
+  if (route_tc_supported(nseq, T, H, L, B))
+    return cuda_status(launch_route_tc(q, w, k, k_pool, pos, nseq, T, H, L, B, h, heads, E,
+                                       ws_region(ws, 0), status_word(ws), (cudaStream_t)stream));
   const int nchunk = (int)((M + kRouteChunk - 1) / kRouteChunk);
   const size_t part_bytes = align256(rows * nchunk * H * sizeof(float));
   return cuda_status(launch_route(q, w, k, k_pool, pos, nseq, T, H, L, B, h, heads, E,

@@ -34,6 +34,16 @@ cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
                          int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
                          int nchunk, int* counters, int* status, cudaStream_t st);
 
+// K2 -- router on tcgen05 for sequences with many queries (route_tc.cu): the full-block
+// part of Eq. (7) as a GEMM against the sequence's pooled keys (bf16 hi + lo), the partial
+// block on CUDA cores, then the top-h.  needs route_tc_ws_bytes(...) of scratch.
+bool route_tc_supported(int nseq, int T, int H, int64_t L, int B);
+size_t route_tc_ws_bytes(int nseq, int T, int H);
+cudaError_t launch_route_tc(const uint16_t* q, const float* w, const uint16_t* k,
+                            const float* k_pool, const int32_t* pos, int nseq, int T, int H,
+                            int64_t L, int B, int h, int32_t* heads, float* E, void* scratch,
+                            int* status, cudaStream_t st);
+
 // K4 -- token scoring on CUDA cores, any head subset (score_simt.cu).
 //   heads == nullptr: all H heads (dense, Eq. 1); otherwise hsel heads per row (Eq. 9).
 //   gather_ids != nullptr: score the tokens gather_ids[row, 0 .. gather_len[row]) instead

@@ -145,6 +145,32 @@ __device__ void select_row_global(const float* __restrict__ x, const int32_t* __
   __syncthreads();
 }
 
+// Block-wide exclusive prefix sum for NT threads (all threads must call).
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan_nt(uint32_t v, uint32_t* warp_sums,
+                                                       uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = NT / 32;
+  uint32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t x = warp_sums[w];
+    if (w < warp) base += x;
+    tot += x;
+  }
+  total = tot;
+  __syncthreads();
+  return base + incl - v;
+}
+
 __global__ void __launch_bounds__(kThreads) topk_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
@@ -532,6 +558,202 @@ __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
   write_row(sel, n, topk, row, idx, vals);
 }
 
+// ---------------------------------------------------------------- row-resident form
+// Rows of up to kRowCap scores and k <= kRowCandCap: one CTA of kSelThreads threads per
+// row keeps the row's keys in shared memory, finds the cutoff bin with a shared-memory
+// histogram of the top kScoreHistBits key bits, compacts the candidates (bins at or above
+// it) and sorts them with the counting sort.  A crowded cutoff falls back to an exact
+// radix select over the resident keys.
+constexpr int kRowCap = 16384;
+constexpr int kRowCandCap = 3072;   // keeps two CTAs per SM
+constexpr int kRowLoadUnroll = 8;
+
+__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_t* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicMin(&red[0], lo);
+    atomicMax(&red[1], hi);
+  }
+  __syncthreads();
+  lo = red[0];
+  hi = red[1];
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2) topk_row_kernel(
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
+    int32_t* __restrict__ idx, float* __restrict__ vals, int64_t row0) {
+  extern __shared__ uint64_t rbuf[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(rbuf);          // [kRowCap] keys, then
+  uint64_t* sorted = rbuf;                                     //   [kRowCandCap] sorted pairs
+  uint64_t* cand = rbuf + kRowCap / 2;                         // [kRowCandCap] candidates
+  __shared__ __align__(16) uint32_t hist[kSubBucketWords];     // histogram, then buckets
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t red[2];
+  __shared__ uint32_t s_cut, s_total, s_big, s_fill, s_flag, s_digit, s_above, s_top;
+  const int t = threadIdx.x, lane = t & 31;
+  const int64_t row = row0 + blockIdx.x;
+  const int n = gather_len ? gather_len[row] : prefix_len(pos, row, L, nullptr);
+  const uint32_t target = (uint32_t)min(n, topk);
+  const float* x = scores + row * stride;
+  const int32_t* imap = index_map ? index_map + row * stride : nullptr;
+
+  for (int b = t; b < kScoreHistBins; b += kSelThreads) hist[b] = 0;
+  if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; s_fill = 0; s_top = 0; }
+  for (int base = 0; base < n; base += kSelThreads * kRowLoadUnroll) {
+    float v[kRowLoadUnroll];
+#pragma unroll
+    for (int j = 0; j < kRowLoadUnroll; ++j) {
+      const int e = base + j * kSelThreads + t;
+      v[j] = e < n ? x[e] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kRowLoadUnroll; ++j) {
+      const int e = base + j * kSelThreads + t;
+      if (e < n) keys[e] = score_key(v[j]);
+    }
+  }
+  __syncthreads();
+  uint32_t cut, btop, C;
+  if ((uint32_t)n <= (uint32_t)kRowCandCap) {
+    // every score is a candidate
+    uint32_t lo = 0xffffffffu, hi = 0;
+    for (int e = t; e < n; e += kSelThreads) {
+      const uint32_t b = keys[e] >> (32 - kScoreHistBits);
+      lo = min(lo, b);
+      hi = max(hi, b);
+    }
+    block_minmax(lo, hi, red);
+    cut = lo;
+    btop = hi;
+    C = (uint32_t)n;
+  } else {
+    for (int e = t; e < n; e += kSelThreads) atomicAdd(&hist[keys[e] >> (32 - kScoreHistBits)], 1u);
+    __syncthreads();
+    HistView<kSelThreads> hv;
+    cut = hist_cutoff<kSelThreads>(hist, target, hv, warp_sums, s_cut, s_total, s_big);
+    // highest occupied bin
+    uint32_t top = 0;
+#pragma unroll
+    for (int i = HistView<kSelThreads>::kPer - 1; i >= 0; --i)
+      if (hv.c[i]) top = max(top, (uint32_t)(hv.hi - 1 - i));
+    if (top) atomicMax(&s_top, top);
+    __syncthreads();
+    btop = s_top;
+    C = s_total;
+  }
+  __syncthreads();
+  const bool fits = C <= (uint32_t)kRowCandCap;
+  if (fits) {
+    for (int base = 0; base < n; base += kSelThreads) {
+      const int e = base + t;
+      const uint32_t key = e < n ? keys[e] : 0u;
+      const bool take = e < n && (key >> (32 - kScoreHistBits)) >= cut;
+      const uint32_t m = __ballot_sync(0xffffffffu, take);
+      uint32_t wb = 0;
+      if (lane == 0 && m) wb = atomicAdd(&s_fill, (uint32_t)__popc(m));
+      wb = __shfl_sync(0xffffffffu, wb, 0);
+      if (take) cand[wb + __popc(m & ((1u << lane) - 1u))] = compose(key, imap ? imap[e] : e);
+    }
+  } else {
+    // crowded cutoff bin: exact threshold by a radix select over the resident keys, then
+    // exactly `target` pairs (above the threshold, then equal ones in index order)
+    uint32_t prefix = 0, mask = 0, kneed = target;
+    for (int p = 0; p < 3; ++p) {
+      const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+      const int nb = p == 2 ? 1024 : 2048;
+      for (int b = t; b < 2048; b += kSelThreads) hist[b] = 0;
+      __syncthreads();
+      for (int e = t; e < n; e += kSelThreads) {
+        const uint32_t key = keys[e];
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+      }
+      __syncthreads();
+      // suffix scan: thread t covers bins nb-1-8t .. nb-8t (8 bins each)
+      uint32_t cb[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int b = nb - 1 - 8 * t - i;
+        cb[i] = b >= 0 ? hist[b] : 0u;
+        local += cb[i];
+      }
+      uint32_t tot;
+      const uint32_t excl = block_excl_scan_nt<kSelThreads>(local, warp_sums, tot);
+      uint32_t run = excl;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (run < kneed && kneed <= run + cb[i]) {
+          s_digit = nb - 1 - 8 * t - i;
+          s_above = run;
+        }
+        run += cb[i];
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= (uint32_t)(nb - 1) << shift;
+      kneed -= s_above;
+      __syncthreads();
+    }
+    const uint32_t thr = prefix;
+    uint32_t eq_taken = 0;
+    for (int base = 0; base < n; base += kSelThreads) {
+      const int e = base + t;
+      const uint32_t key = e < n ? keys[e] : 0u;
+      const bool gt = e < n && key > thr;
+      const bool eq = e < n && key == thr;
+      uint32_t tot;
+      const uint32_t ex =
+          block_excl_scan_nt<kSelThreads>((gt ? 1u << 16 : 0u) | (eq ? 1u : 0u), warp_sums, tot);
+      const uint32_t re = eq_taken + (ex & 0xffffu);
+      const bool take = gt || (eq && re < kneed);
+      const uint32_t m = __ballot_sync(0xffffffffu, take);
+      uint32_t wb = 0;
+      if (lane == 0 && m) wb = atomicAdd(&s_fill, (uint32_t)__popc(m));
+      wb = __shfl_sync(0xffffffffu, wb, 0);
+      if (take) cand[wb + __popc(m & ((1u << lane) - 1u))] = compose(key, imap ? imap[e] : e);
+      eq_taken += tot & 0xffffu;
+    }
+    C = target;
+    cut = thr >> (32 - kScoreHistBits);
+    btop = 0;
+    for (int e = t; e < n; e += kSelThreads) btop = max(btop, keys[e] >> (32 - kScoreHistBits));
+    uint32_t lo_dummy = 0xffffffffu;
+    if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; }
+    __syncthreads();
+    block_minmax(lo_dummy, btop, red);
+  }
+  __syncthreads();
+  // keys are dead from here on: their space holds the sorted pairs
+  if (!group_sort_desc<kSelThreads>(cand, C, sorted, hist, cut, btop, warp_sums, s_flag)) {
+    int sortn = kSelThreads;
+    while ((uint32_t)sortn < C) sortn <<= 1;
+    for (int i = t; i < sortn; i += kSelThreads) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
+    __syncthreads();
+    switch (sortn / kSelThreads) {   // C <= kRowCandCap <= 16 * kSelThreads
+      case 1: sort_buf_desc_e<1, kSelThreads>(sorted); break;
+      case 2: sort_buf_desc_e<2, kSelThreads>(sorted); break;
+      case 4: sort_buf_desc_e<4, kSelThreads>(sorted); break;
+      case 8: sort_buf_desc_e<8, kSelThreads>(sorted); break;
+      default: sort_buf_desc_e<16, kSelThreads>(sorted); break;
+    }
+  }
+  for (int i = t; i < topk; i += kSelThreads) {
+    const int64_t o = row * topk + i;
+    if ((uint32_t)i < target) {
+      const uint64_t v = sorted[i];
+      idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
+      if (vals) vals[o] = key_score((uint32_t)(v >> 32));
+    } else {
+      idx[o] = -1;
+      if (vals) vals[o] = __int_as_float(0xff800000);
+    }
+  }
+}
+
 }  // namespace
 
 int topk_sort_size(int topk) {
@@ -588,6 +810,20 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
   (void)status;
   const int sortn = topk_sort_size(topk);
   const int64_t maxlen = gather_len ? stride : L;
+  if (maxlen <= kRowCap && topk <= kRowCandCap) {
+    const size_t smem = (size_t)(kRowCap / 2 + kRowCandCap) * sizeof(uint64_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_row_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
+      const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
+      topk_row_kernel<<<(unsigned)nr, kSelThreads, smem, st>>>(scores, stride, pos, L, gather_len,
+                                                               index_map, topk, idx, vals, row0);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   const int G = cluster_size_for(maxlen, sortn);
   if (G > 0) {
     const int64_t slice = (((maxlen + G - 1) / G) + 3) & ~int64_t(3);

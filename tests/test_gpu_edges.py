@@ -48,6 +48,9 @@ CASES = {
     "B_larger_than_L": dict(B=1024, L=300),
     "many_rows": dict(nseq=3, T=150, L=700, topk=50, kprime=100),
     "max_topk": dict(nseq=1, T=2, L=20000, topk=16384, kprime=16384, B=128),
+    # many queries per sequence: tensor-core router and query-block scorer
+    "blocks_two_seqs_H16": dict(nseq=2, T=64, L=1000, H=16, h=4, topk=64, kprime=128),
+    "blocks_H64_B32": dict(nseq=1, T=40, L=3000, H=64, h=8, B=32, topk=128, kprime=256),
 }
 
 

@@ -406,9 +406,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override an integer field of the workload (e.g. T=8192), for "
+                         "smaller profiling runs; the JSON line names the result")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = WORKLOADS[args.workload]
+    for kv in args.set:
+        field, value = kv.split("=", 1)
+        wl = wl.replace(**{field: int(value)})
+    if args.set:
+        wl = wl.replace(name=wl.name + "[" + ",".join(args.set) + "]")
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_cuda(args, wl)

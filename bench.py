@@ -121,6 +121,19 @@ def block_form(wl) -> bool:
     return wl.T >= 256 // hs and wl.T >= 16
 
 
+def misa_step_launches(wl) -> int:
+    """Kernels one MISA step launches, following the library's dispatch: pooling, the router
+    (one kernel on CUDA cores, or four on tensor cores for many queries per sequence), the
+    scorer's gather/offsets kernel and the scorer, then the top-k (histogram path for long
+    decode rows: two kernels, three above k = 4096; otherwise one)."""
+    n = 1 + (4 if (128 % wl.H == 0 and wl.T >= 4 * (128 // wl.H) and -(-wl.L // wl.B) <= 256)
+             else 1)
+    n += 2
+    hist_path = wl.rows <= 1024 and wl.L >= 8192 and not block_form(wl)
+    n += (2 + (wl.topk > 4096)) if hist_path else 1
+    return n
+
+
 def algorithmic_flops_score(wl) -> float:
     """Multiply-add work of Eq. (9) over every causal (query, key) pair: 2 * h * d each."""
     return 2.0 * wl.h * wl.d * wl.query_prefix_tokens()
@@ -362,6 +375,7 @@ def run_cuda(args, wl):
                     "peak_source": peaks["source"] + " HBM copy",
                     "algorithmic_bytes": score_bytes, "avg_ms": ms_score_kernel}
 
+    launches_per_step = misa_step_launches(wl)
     line = {
         "metric": METRIC, "value": units * world / (ms_misa * 1e-3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_misa,
@@ -385,7 +399,7 @@ def run_cuda(args, wl):
         },
         "e2e": {"value": units * world / (ms_e2e * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if world > 1:

@@ -169,15 +169,30 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // last CTA of this row: E[j] = |w_j| / M * sum over chunks, then the top-h heads
-  if (tid < H) {
-    float sum = 0.f;
-    for (int c = 0; c < nch; ++c) sum += __ldcg(partial + (row * nchunk + c) * H + tid);
-    const float v = fabsf(w[row * H + tid]) * sum / (float)M;
-    ev[tid] = v;
-    if (E) E[row * H + tid] = v;
+  // last CTA of this row: E[j] = |w_j| / M * sum over chunks, then the top-h heads.  The
+  // chunk partials are summed by all threads (kRouteThreads / 32 groups of 32 heads), so
+  // their L2 loads are in flight together rather than one after another.
+  constexpr int kGroups = kRouteThreads / 32;
+  {
+    const int jj = tid & 31, grp = tid >> 5;
+    for (int j0 = 0; j0 < H; j0 += 32) {
+      const int j = j0 + jj;
+      float sum = 0.f;
+      if (j < H)
+        for (int c = grp; c < nch; c += kGroups) sum += __ldcg(partial + (row * nchunk + c) * H + j);
+      red[grp][jj] = sum;
+      __syncthreads();
+      if (grp == 0 && j < H) {
+        float tot = 0.f;
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) tot += red[g][jj];
+        const float v = fabsf(w[row * H + j]) * tot / (float)M;
+        ev[j] = v;
+        if (E) E[row * H + j] = v;
+      }
+      __syncthreads();
+    }
   }
-  __syncthreads();
   if (tid < 32) select_top_h(ev, H, h, heads + row * h);
 }
 

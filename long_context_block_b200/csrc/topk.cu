@@ -63,88 +63,6 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
   return base + incl - v;
 }
 
-// Write the first min(n, topk) sorted pairs of `sel` as (index, value), pad the rest.
-__device__ __forceinline__ void write_row(const uint64_t* sel, int n, int topk, int64_t row,
-                                          int32_t* idx, float* vals) {
-  const int nvalid = n < topk ? n : topk;
-  for (int i = threadIdx.x; i < topk; i += kThreads) {
-    const int64_t o = row * topk + i;
-    if (i < nvalid) {
-      const uint64_t v = sel[i];
-      idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
-      if (vals) vals[o] = key_score((uint32_t)(v >> 32));
-    } else {
-      idx[o] = -1;
-      if (vals) vals[o] = __int_as_float(0xff800000);
-    }
-  }
-}
-
-// Exact selection over a row in global memory (three radix passes that re-read the row):
-// fills sel[0 .. sortn) with the min(n, topk) selected (key, index) pairs and zero padding.
-// All threads of the block must call it.
-__device__ void select_row_global(const float* __restrict__ x, const int32_t* __restrict__ imap,
-                                  int n, int topk, int sortn, uint64_t* sel, uint32_t* hist,
-                                  uint32_t* warp_sums, uint32_t& s_digit, uint32_t& s_above,
-                                  uint32_t& s_cnt) {
-  const int tid = threadIdx.x;
-  if (n <= topk) {
-    for (int i = tid; i < sortn; i += kThreads)
-      sel[i] = i < n ? compose(score_key(x[i]), imap ? imap[i] : i) : 0ull;
-  } else {
-    uint32_t prefix = 0, mask = 0, kneed = (uint32_t)topk;
-    for (int p = 0; p < 3; ++p) {
-      const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
-      const int nb = p == 2 ? 1024 : 2048;
-      for (int b = tid; b < kBins; b += kThreads) hist[b] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += kThreads) {
-        const uint32_t key = score_key(x[i]);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-      }
-      __syncthreads();
-      // suffix scan: thread t covers bins nb-1-2t (hi) and nb-2-2t (lo)
-      const bool act = 2 * tid < nb;
-      const uint32_t c_hi = act ? hist[nb - 1 - 2 * tid] : 0u;
-      const uint32_t c_lo = act ? hist[nb - 2 - 2 * tid] : 0u;
-      uint32_t total;
-      const uint32_t excl = block_excl_scan(c_hi + c_lo, warp_sums, total);
-      if (act) {
-        if (excl < kneed && kneed <= excl + c_hi) {
-          s_digit = nb - 1 - 2 * tid;
-          s_above = excl;
-        } else if (excl + c_hi < kneed && kneed <= excl + c_hi + c_lo) {
-          s_digit = nb - 2 - 2 * tid;
-          s_above = excl + c_hi;
-        }
-      }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      mask |= (uint32_t)(nb - 1) << shift;
-      kneed -= s_above;
-      __syncthreads();
-    }
-    const uint32_t thr = prefix;
-    if (tid == 0) s_cnt = 0;
-    __syncthreads();
-    uint32_t eq_taken = 0;
-    for (int base = 0; base < n; base += kThreads) {
-      const int i = base + tid;
-      const uint32_t key = i < n ? score_key(x[i]) : 0u;
-      const bool gt = i < n && key > thr;
-      const bool eq = i < n && key == thr;
-      if (gt) sel[atomicAdd(&s_cnt, 1u)] = compose(key, imap ? imap[i] : i);
-      uint32_t total;
-      const uint32_t rank = block_excl_scan(eq ? 1u : 0u, warp_sums, total);
-      if (eq && eq_taken + rank < kneed) sel[atomicAdd(&s_cnt, 1u)] = compose(key, imap ? imap[i] : i);
-      eq_taken += total;
-    }
-    __syncthreads();
-    for (int i = topk + tid; i < sortn; i += kThreads) sel[i] = 0ull;
-  }
-  __syncthreads();
-}
-
 // Block-wide exclusive prefix sum for NT threads (all threads must call).
 template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan_nt(uint32_t v, uint32_t* warp_sums,
@@ -169,6 +87,106 @@ __device__ __forceinline__ uint32_t block_excl_scan_nt(uint32_t v, uint32_t* war
   total = tot;
   __syncthreads();
   return base + incl - v;
+}
+
+// Write the first min(n, topk) sorted pairs of `sel` as (index, value), pad the rest.
+__device__ __forceinline__ void write_row(const uint64_t* sel, int n, int topk, int64_t row,
+                                          int32_t* idx, float* vals) {
+  const int nvalid = n < topk ? n : topk;
+  for (int i = threadIdx.x; i < topk; i += kThreads) {
+    const int64_t o = row * topk + i;
+    if (i < nvalid) {
+      const uint64_t v = sel[i];
+      idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
+      if (vals) vals[o] = key_score((uint32_t)(v >> 32));
+    } else {
+      idx[o] = -1;
+      if (vals) vals[o] = __int_as_float(0xff800000);
+    }
+  }
+}
+
+// Exact selection over a row in global memory (three radix passes that re-read the row):
+// fills sel[0 .. sortn) with the min(n, topk) selected (key, index) pairs and zero padding.
+// All threads of the block must call it.
+// Exact selection over a row in global memory (three radix passes that re-read the row):
+// fills sel[0 .. sortn) with the min(n, topk) selected (key, index) pairs and zero padding.
+// All NT threads of the block must call it.
+template <int NT>
+__device__ void select_row_global_nt(const float* __restrict__ x, const int32_t* __restrict__ imap,
+                                     int n, int topk, int sortn, uint64_t* sel, uint32_t* hist,
+                                     uint32_t* warp_sums, uint32_t& s_digit, uint32_t& s_above,
+                                     uint32_t& s_cnt) {
+  const int tid = threadIdx.x;
+  constexpr int kPerT = kBins / NT;   // histogram bins per thread in the digit search
+  if (n <= topk) {
+    for (int i = tid; i < sortn; i += NT)
+      sel[i] = i < n ? compose(score_key(x[i]), imap ? imap[i] : i) : 0ull;
+  } else {
+    uint32_t prefix = 0, mask = 0, kneed = (uint32_t)topk;
+    for (int p = 0; p < 3; ++p) {
+      const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+      const int nb = p == 2 ? 1024 : 2048;
+      for (int b = tid; b < kBins; b += NT) hist[b] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += NT) {
+        const uint32_t key = score_key(x[i]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+      }
+      __syncthreads();
+      // suffix scan: thread t covers bins nb-1-kPerT*t-i, i < kPerT
+      uint32_t cb[kPerT], local = 0;
+#pragma unroll
+      for (int i = 0; i < kPerT; ++i) {
+        const int b = nb - 1 - kPerT * tid - i;
+        cb[i] = b >= 0 ? hist[b] : 0u;
+        local += cb[i];
+      }
+      uint32_t total;
+      const uint32_t excl = block_excl_scan_nt<NT>(local, warp_sums, total);
+      uint32_t run = excl;
+#pragma unroll
+      for (int i = 0; i < kPerT; ++i) {
+        if (run < kneed && kneed <= run + cb[i]) {
+          s_digit = nb - 1 - kPerT * tid - i;
+          s_above = run;
+        }
+        run += cb[i];
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= (uint32_t)(nb - 1) << shift;
+      kneed -= s_above;
+      __syncthreads();
+    }
+    const uint32_t thr = prefix;
+    if (tid == 0) s_cnt = 0;
+    __syncthreads();
+    uint32_t eq_taken = 0;
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + tid;
+      const uint32_t key = i < n ? score_key(x[i]) : 0u;
+      const bool gt = i < n && key > thr;
+      const bool eq = i < n && key == thr;
+      if (gt) sel[atomicAdd(&s_cnt, 1u)] = compose(key, imap ? imap[i] : i);
+      uint32_t total;
+      const uint32_t rank = block_excl_scan_nt<NT>(eq ? 1u : 0u, warp_sums, total);
+      if (eq && eq_taken + rank < kneed) sel[atomicAdd(&s_cnt, 1u)] = compose(key, imap ? imap[i] : i);
+      eq_taken += total;
+    }
+    __syncthreads();
+    for (int i = topk + tid; i < sortn; i += NT) sel[i] = 0ull;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void select_row_global(const float* __restrict__ x,
+                                                  const int32_t* __restrict__ imap, int n, int topk,
+                                                  int sortn, uint64_t* sel, uint32_t* hist,
+                                                  uint32_t* warp_sums, uint32_t& s_digit,
+                                                  uint32_t& s_above, uint32_t& s_cnt) {
+  select_row_global_nt<kThreads>(x, imap, n, topk, sortn, sel, hist, warp_sums, s_digit, s_above,
+                                 s_cnt);
 }
 
 __global__ void __launch_bounds__(kThreads) topk_kernel(
@@ -465,12 +483,14 @@ __global__ void __launch_bounds__(kSelThreads) topk_scatter_kernel(
 
 // Pass 2: CTA g of a row sorts group g's candidates and writes them at their positions.
 __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
-    const int32_t* __restrict__ pos, int64_t L, const uint32_t* __restrict__ hist, int topk,
-    const uint64_t* __restrict__ cand, int32_t* __restrict__ idx, float* __restrict__ vals) {
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    const uint32_t* __restrict__ hist, int topk, const uint64_t* __restrict__ cand,
+    int32_t* __restrict__ idx, float* __restrict__ vals) {
   extern __shared__ uint64_t gbuf[];   // [2 * kGroupBuf]: gathered, then sorted
   __shared__ uint32_t buckets[kSubBucketWords];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t s_cut, s_total, s_big, s_lo, s_hi, s_start, s_cnt, s_flag;
+  __shared__ uint32_t s_digit, s_above, s_sel;
   uint64_t* gathered = gbuf;
   uint64_t* sorted = gbuf + kGroupBuf;
   const int t = threadIdx.x;
@@ -482,7 +502,34 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
   HistView<kSelThreads> hv;
   const uint32_t cut = hist_cutoff<kSelThreads>(hist + row * kScoreHistBins, target, hv, warp_sums,
                                                 s_cut, s_total, s_big);
-  if (hist_overflow(s_total, s_big)) return;   // topk_hist_overflow_kernel takes this row
+  if (hist_overflow(s_total, s_big)) {
+    // crowded cutoff (e.g. many equal scores): an exact selection over the whole row, here
+    // by CTA 0 when the selected pairs fit its buffer, else by topk_hist_overflow_kernel
+    if (g != 0 || topk > kGroupBuf) return;
+    int sortn = kSelThreads;
+    while (sortn < topk) sortn <<= 1;
+    select_row_global_nt<kSelThreads>(scores + row * stride, nullptr, n, topk, sortn, gbuf, buckets,
+                                      warp_sums, s_digit, s_above, s_sel);
+    switch (sortn / kSelThreads) {
+      case 1: sort_buf_desc_e<1, kSelThreads>(gbuf); break;
+      case 2: sort_buf_desc_e<2, kSelThreads>(gbuf); break;
+      case 4: sort_buf_desc_e<4, kSelThreads>(gbuf); break;
+      case 8: sort_buf_desc_e<8, kSelThreads>(gbuf); break;
+      default: sort_buf_desc_e<16, kSelThreads>(gbuf); break;
+    }
+    for (int i = t; i < topk; i += kSelThreads) {
+      const int64_t o = row * topk + i;
+      if ((uint32_t)i < target) {
+        const uint64_t v = gbuf[i];
+        idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
+        if (vals) vals[o] = key_score((uint32_t)(v >> 32));
+      } else {
+        idx[o] = -1;
+        if (vals) vals[o] = __int_as_float(0xff800000);
+      }
+    }
+    return;
+  }
   {
     uint32_t run = hv.before, lo = 0xffffffffu, hb = 0, cnt = 0, st = 0xffffffffu;
 #pragma unroll
@@ -537,7 +584,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
   }
 }
 
-// Exact selection for the rows topk_group_kernel leaves out (same overflow test).
+// Exact selection for the rows topk_group_kernel leaves out (same overflow test, k > 4096).
 __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const uint32_t* __restrict__ hist, int topk, int sortn, int32_t* __restrict__ idx,
@@ -775,9 +822,9 @@ cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t*
                            (int)smem);
   if (e != cudaSuccess) return e;
   topk_group_kernel<<<dim3(kMaxGroups, (unsigned)rows), kSelThreads, smem, st>>>(
-      pos, L, hist, topk, cand, idx, vals);
+      scores, stride, pos, L, hist, topk, cand, idx, vals);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || topk <= kGroupBuf) return e;   // the group kernel covers overflow rows
   const int sortn = topk_sort_size(topk);
   const size_t ov_smem = (size_t)sortn * sizeof(uint64_t);
   e = cudaFuncSetAttribute(topk_hist_overflow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

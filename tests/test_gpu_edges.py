@@ -159,3 +159,20 @@ def test_score_rows_entry_point(M, T, pos_mode):
                             what=f"routed {n},{t}")
             tl.check_scores(dense[n, t, :P], orc.dense_scores(q_t, w_t, kk, P),
                             what=f"dense {n},{t}")
+
+
+def test_tied_long_rows_exact_fallback(M):
+    """Rows long enough for the histogram top-k whose scores are all equal: the crowded
+    cutoff takes the exact fallback (inside the group kernel for k <= 4096, the separate
+    overflow kernel above) and returns the lowest indices."""
+    wl = _wl(nseq=2, T=1, L=10000, H=8, h=3, topk=2048, kprime=8192)
+    x = make_inputs(wl, seed=5)
+    x.k_bits[:] = fp32_to_bf16_bits(np.full((128,), 0.05, dtype=np.float32))[None, None, :]
+    q, w, k, pos = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, wl.B)
+    heads = M.misa_route_heads(q, w, k, kp, pos, wl.B, wl.h)
+    for kk in (wl.topk, wl.kprime):
+        idx = M.misa_score_topk(q, w, k, heads, pos, kk, return_vals=False)
+        didx = M.dsa_score_topk(q, w, k, pos, kk, return_vals=False)
+        ref = torch.arange(kk, dtype=torch.int32).expand(2, 1, kk)
+        assert torch.equal(idx.cpu(), ref) and torch.equal(didx.cpu(), ref), kk

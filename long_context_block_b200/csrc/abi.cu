@@ -103,10 +103,10 @@ size_t score_ws(int nseq, int T, int64_t L, int nh) {
   return kStatusBytes + align256((size_t)rows * L * sizeof(float)) +
          score_tc_ws_bytes(nseq, T, nh) + (hist_path(nseq, T, L, nh) ? hist_path_bytes(rows) : 0);
 }
-size_t dagger_ws(int nseq, int T, int kprime) {
+size_t dagger_ws(int nseq, int T, int H, int kprime) {
   const size_t rows = (size_t)nseq * T;
   return kStatusBytes + 2 * align256(rows * kprime * sizeof(int32_t)) +
-         align256(rows * sizeof(int32_t));
+         align256(rows * sizeof(int32_t)) + score_tc_ws_bytes(nseq, T, H, true);
 }
 
 int check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -139,7 +139,7 @@ size_t misa_workspace_size(int op, int nseq, int T, int H, int d, int64_t L, int
       return kStatusBytes + score_tc_ws_bytes(nseq, T, h);
     case MISA_OP_DAGGER_RERANK:
       if (check_topk(topk) != MISA_OK || kprime < topk || kprime > MISA_MAX_TOPK) return 0;
-      return dagger_ws(nseq, T, kprime);
+      return dagger_ws(nseq, T, H, kprime);
     default:
       return 0;
   }
@@ -287,17 +287,22 @@ int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k, con
   MISA_TRY(check_dev(cand, rows * kprime * 4, 4));
   MISA_TRY(check_dev(idx, rows * topk * 4, 4));
   MISA_TRY(check_opt(vals, rows * topk * 4, 4));
-  MISA_TRY(check_ws(ws, ws_bytes, dagger_ws(nseq, T, kprime)));
+  MISA_TRY(check_ws(ws, ws_bytes, dagger_ws(nseq, T, H, kprime)));
   cudaStream_t st = (cudaStream_t)stream;
   int* status = status_word(ws);
   const size_t ids_bytes = align256(rows * kprime * sizeof(int32_t));
   int32_t* sorted = reinterpret_cast<int32_t*>(ws_region(ws, 0));
   float* cscore = reinterpret_cast<float*>(ws_region(ws, ids_bytes));
   int32_t* count = reinterpret_cast<int32_t*>(ws_region(ws, 2 * ids_bytes));
+  void* tc_scratch = ws_region(ws, 2 * ids_bytes + align256(rows * sizeof(int32_t)));
   MISA_TRY(cuda_status(
       launch_sort_candidates(cand, pos, (int)rows, L, kprime, sorted, count, status, st)));
-  MISA_TRY(cuda_status(launch_score_simt(q, w, k, nullptr, H, pos, sorted, count, nseq, T, H, L,
-                                         cscore, kprime, status, st)));
+  if (score_tc_supported(nseq, T, H, L, kprime))
+    MISA_TRY(cuda_status(launch_score_tc(q, w, k, nullptr, H, pos, nseq, T, H, L, cscore, kprime,
+                                         tc_scratch, status, nullptr, st, sorted, count)));
+  else
+    MISA_TRY(cuda_status(launch_score_simt(q, w, k, nullptr, H, pos, sorted, count, nseq, T, H,
+                                           L, cscore, kprime, status, st)));
   return cuda_status(launch_topk(cscore, kprime, pos, L, count, sorted, (int)rows, topk, idx,
                                  vals, status, st));
 }

@@ -56,17 +56,23 @@ cudaError_t launch_score_simt(const uint16_t* q, const float* w, const uint16_t*
 
 // K4 -- token scoring on tcgen05 tensor cores (score_tc.cu): rows streaming their own key
 // prefix (decode form), or blocks of queries sharing key tiles (block form, when a
-// sequence has enough queries).  Same contract as launch_score_simt without the gather
-// mode; needs score_tc_ws_bytes(nseq, T, nh) bytes of 256-aligned scratch.
-bool score_tc_supported(int nseq, int T, int nh, int64_t L);
+// sequence has enough queries).  Same contract as launch_score_simt; needs
+// score_tc_ws_bytes(nseq, T, nh, gather) bytes of 256-aligned scratch.
+//   span: 0 for prefix scoring, else the gather list stride (kprime).
+bool score_tc_supported(int nseq, int T, int nh, int64_t L, int64_t span = 0);
 bool score_tc_block_form(int nh, int T);
-size_t score_tc_ws_bytes(int nseq, int T, int nh);
+size_t score_tc_ws_bytes(int nseq, int T, int nh, bool gather = false);
 //   hist (nullable, zeroed by the caller): per-row kScoreHistBins-bin histogram of the
-//   written scores' keys, accumulated in the epilogue.
+//   written scores' keys, accumulated in the epilogue (prefix decode form only).
+//   gather_ids / gather_len (both or neither): row r scores the gather_len[r] tokens
+//   gather_ids[r * out_stride + i] (each in [0, L)) into out[r * out_stride + i]; every
+//   row takes the decode form and its keys are fetched four rows per TMA gather.
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
-                            int* status, uint32_t* hist, cudaStream_t st);
+                            int* status, uint32_t* hist, cudaStream_t st,
+                            const int32_t* gather_ids = nullptr,
+                            const int32_t* gather_len = nullptr);
 
 // K5 -- per-row top-k selection (topk.cu).
 //   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.

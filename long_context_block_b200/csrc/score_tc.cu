@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ wsel, const int32_t* __restrict__ pos,
     const int32_t* __restrict__ tile_off, int units, Units geo, int64_t L,
-    float* __restrict__ out, int64_t out_stride, int* status, uint32_t* __restrict__ hist) {
+    float* __restrict__ out, int64_t out_stride, int* status, uint32_t* __restrict__ hist,
+    const int32_t* __restrict__ gidx, const int32_t* __restrict__ glen) {
   using C = Cfg<HS, QB>;
   constexpr int N = C::N;
   constexpr int kEpiThreads = 32 * C::kEpiWarps;
@@ -190,48 +191,71 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // The whole warp walks the loop (waits are polled by lane 0 and broadcast); lane 0
+    // issues the tile loads, or in gather mode every lane gathers four key rows.
     int issued = 0, qissued = 0, wissued = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_q);
-      int u = u_first;
-      Seg sg;
-      bool ok = true;
-      while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
-        const int slot = qissued % C::kQBufs;
-        if (!mbar_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status,
-                       kWaitCycles))
-          break;
-        uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
+    }
+    int u = u_first;
+    Seg sg;
+    bool ok = true;
+    while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
+      const int slot = qissued % C::kQBufs;
+      if (!warp_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status)) break;
+      uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
+      if (lane == 0) {
         mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
         tma_load_2d(qb, &tm_q, &qfull[slot], 0, sg.u * N);
         tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
-        const int wslot = qissued % C::kWBufs;
-        if (!mbar_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status,
-                       kWaitCycles)) {
-          ++qissued;
-          break;
-        }
+      }
+      const int wslot = qissued % C::kWBufs;
+      if (!warp_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status)) {
+        ++qissued;
+        break;
+      }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&wfull[wslot], C::kWBytes);
         bulk_load(base + C::kWBase + wslot * C::kWBytes, wsel + (int64_t)sg.u * N, C::kWBytes,
                   &wfull[wslot]);
-        ++qissued;
-        ++wissued;
-        const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
-        for (int j = sg.a; j < sg.b; ++j) {
-          const int s = issued % C::kStages;
-          if (!mbar_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status,
-                         kWaitCycles)) {
-            ok = false;
-            break;
+      }
+      ++qissued;
+      ++wissued;
+      const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
+      // gather mode (QB == 1, unit = row): the row's token list and its length
+      const int32_t* ids = gidx ? gidx + (int64_t)sg.u * out_stride : nullptr;
+      const int cnt = gidx ? min(max(glen[sg.u], 0), (int)out_stride) : 0;
+      for (int j = sg.a; j < sg.b; ++j) {
+        const int s = issued % C::kStages;
+        int32_t r[4];
+        if (ids) {   // fetch the ids before the wait so their latency hides behind it
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = j * kTileKeys + 4 * lane + i;
+            int32_t id = c < cnt ? ids[c] : 0;   // padding keys are masked by the epilogue
+            if (id < 0 || id >= L) id = 0;
+            r[i] = (int32_t)(y0 + id);
           }
-          uint8_t* kb = base + C::kStageBase + s * kKeyTileBytes;
+        }
+        if (!warp_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* kb = base + C::kStageBase + s * kKeyTileBytes;
+        if (ids) {
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
+          __syncwarp();
+          uint8_t* dst = kb + lane * 4 * 128;   // rows 4*lane .. 4*lane+3 of both halves
+          tma_gather4(dst, &tm_k, &full[s], 0, r[0], r[1], r[2], r[3]);
+          tma_gather4(dst + kKeyHalfBytes, &tm_k, &full[s], 64, r[0], r[1], r[2], r[3]);
+        } else if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
           const int32_t y = (int32_t)(y0 + (int64_t)j * kTileKeys);
           tma_load_2d(kb, &tm_k, &full[s], 0, y);
           tma_load_2d(kb + kKeyHalfBytes, &tm_k, &full[s], 64, y);
-          ++issued;
         }
+        ++issued;
       }
     }
     __syncthreads();   // (A) every role has left its loop
@@ -315,7 +339,9 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 #pragma unroll
       for (int q = 0; q < kQPerWarp; ++q) {
         const int t = tq0 + q0 + q;
-        P[q] = t < geo.T ? prefix_len(pos, (int64_t)n * geo.T + t, L, nullptr) : 0;
+        P[q] = t >= geo.T ? 0
+               : gidx  ? min(max(glen[sg.u], 0), (int)out_stride)
+                       : prefix_len(pos, (int64_t)n * geo.T + t, L, nullptr);
       }
       // this warp's queries are consecutive rows of the output
       float* obase = out + ((int64_t)n * geo.T + min(tq0 + q0, geo.T - 1)) * out_stride;
@@ -381,11 +407,13 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 
 // Gather each unit's head vectors (routed heads, or all heads) into a zero-padded
 // [units, QB * HS, 128] bf16 operand and their weights into [units, QB * HS]; block 0
-// also lays the units' key tiles end to end (tile_off[u] = tiles of units < u).
+// also lays the units' key tiles end to end (tile_off[u] = tiles of units < u), sized by
+// the causal prefix or, in gather mode, by the row's token-list length.
 __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
     const uint16_t* __restrict__ q, const float* __restrict__ w, const int32_t* __restrict__ heads,
     int hsel, int H, int HS, Units geo, const int32_t* __restrict__ pos, int units, int64_t L,
-    uint4* __restrict__ qg, float* __restrict__ wg, int32_t* __restrict__ tile_off, int* status) {
+    const int32_t* __restrict__ glen, int gmax, uint4* __restrict__ qg, float* __restrict__ wg,
+    int32_t* __restrict__ tile_off, int* status) {
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   const int nh = heads ? hsel : H;
@@ -420,8 +448,11 @@ __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
       if (uu < units) {
         const int nn = geo.seq(uu), ta = geo.t0(uu);
         int Pmax = 0;
-        for (int qq = 0; qq < geo.QB && ta + qq < geo.T; ++qq)
-          Pmax = max(Pmax, prefix_len(pos, (int64_t)nn * geo.T + ta + qq, L, status));
+        if (glen)   // gather mode: one row per unit, its token-list length
+          Pmax = min(max(glen[uu], 0), gmax);
+        else
+          for (int qq = 0; qq < geo.QB && ta + qq < geo.T; ++qq)
+            Pmax = max(Pmax, prefix_len(pos, (int64_t)nn * geo.T + ta + qq, L, status));
         v = (Pmax + kTileKeys - 1) / kTileKeys;
       }
       int incl = v;
@@ -490,7 +521,7 @@ template <int HS, int QB>
 cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float* wg,
                        const int32_t* pos, const int32_t* tile_off, int units, Units geo,
                        int64_t L, float* out, int64_t out_stride, int* status, uint32_t* hist,
-                       cudaStream_t st) {
+                       const int32_t* gidx, const int32_t* glen, cudaStream_t st) {
   using C = Cfg<HS, QB>;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -499,7 +530,7 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   score_tc_kernel<HS, QB><<<sms, C::kThreads, C::kSmemBytes, st>>>(
-      tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist);
+      tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist, gidx, glen);
   return cudaGetLastError();
 }
 
@@ -508,12 +539,13 @@ struct Plan {
   int HS, QB, N;
 };
 
-Plan plan_for(int nh, int T) {
+Plan plan_for(int nh, int T, bool gather = false) {
   Plan p;
-  // block form when a sequence has enough queries to fill a 256-column B operand
+  // block form when a sequence has enough queries to fill a 256-column B operand (rows
+  // with their own token lists always take the decode form)
   const int hs_pow2 = nh <= 8 ? 8 : nh <= 16 ? 16 : nh <= 32 ? 32 : nh <= 64 ? 64 : 128;
   const int qb = 256 / hs_pow2;
-  if (T >= qb && T >= 16) {
+  if (!gather && T >= qb && T >= 16) {
     p.HS = hs_pow2;
     p.QB = qb;
   } else {
@@ -526,8 +558,8 @@ Plan plan_for(int nh, int T) {
 
 }  // namespace
 
-size_t score_tc_ws_bytes(int nseq, int T, int nh) {
-  const Plan p = plan_for(nh, T);
+size_t score_tc_ws_bytes(int nseq, int T, int nh, bool gather) {
+  const Plan p = plan_for(nh, T, gather);
   const int64_t units = (int64_t)nseq * ((T + p.QB - 1) / p.QB);
   return align256((size_t)units * p.N * kHeadDim * 2) + align256((size_t)units * p.N * 4) +
          align256((size_t)(units + 1) * 4);
@@ -535,10 +567,10 @@ size_t score_tc_ws_bytes(int nseq, int T, int nh) {
 
 bool score_tc_block_form(int nh, int T) { return plan_for(nh, T).QB > 1; }
 
-bool score_tc_supported(int nseq, int T, int nh, int64_t L) {
-  const Plan p = plan_for(nh, T);
+bool score_tc_supported(int nseq, int T, int nh, int64_t L, int64_t span) {
+  const Plan p = plan_for(nh, T, span > 0);
   const int64_t units = (int64_t)nseq * ((T + p.QB - 1) / p.QB);
-  const int64_t tiles = units * ((L + kTileKeys - 1) / kTileKeys);
+  const int64_t tiles = units * (((span > 0 ? span : L) + kTileKeys - 1) / kTileKeys);
   return nh >= 1 && nh <= 128 && (int64_t)nseq * L < INT32_MAX && tiles < INT32_MAX &&
          units * p.N < INT32_MAX && encode_fn() != nullptr;
 }
@@ -546,9 +578,11 @@ bool score_tc_supported(int nseq, int T, int nh, int64_t L) {
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
-                            int* status, uint32_t* hist, cudaStream_t st) {
+                            int* status, uint32_t* hist, cudaStream_t st, const int32_t* gidx,
+                            const int32_t* glen) {
+  const bool gather = gidx != nullptr;
   const int nh = heads ? hsel : H;
-  const Plan p = plan_for(nh, T);
+  const Plan p = plan_for(nh, T, gather);
   Units geo;
   geo.T = T;
   geo.QB = p.QB;
@@ -560,20 +594,21 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
   float* wg = reinterpret_cast<float*>(c);
   c += align256((size_t)units * p.N * 4);
   int32_t* tile_off = reinterpret_cast<int32_t*>(c);
-  if (p.QB > 1) hist = nullptr;
+  if (p.QB > 1 || gather) hist = nullptr;
 
-  score_tc_prep_kernel<<<units, 1024, 0, st>>>(q, w, heads, hsel, H, p.HS, geo, pos, units, L, qg,
-                                               wg, tile_off, status);
+  score_tc_prep_kernel<<<units, 1024, 0, st>>>(q, w, heads, hsel, H, p.HS, geo, pos, units, L,
+                                               glen, (int)out_stride, qg, wg, tile_off, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // key rows come as whole 128-key tiles, or one row per box for the gather
   CUtensorMap tk, tq;
-  if (!make_map(&tk, k, (uint64_t)nseq * L, kTileKeys) ||
+  if (!make_map(&tk, k, (uint64_t)nseq * L, gather ? 1u : (uint32_t)kTileKeys) ||
       !make_map(&tq, qg, (uint64_t)units * p.N, (uint32_t)p.N))
     return cudaErrorInvalidValue;
 #define MISA_TC_CASE(HS_, QB_)                                                                  \
   if (p.HS == HS_ && p.QB == QB_)                                                               \
     return launch_cfg<HS_, QB_>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, \
-                                hist, st);
+                                hist, gidx, glen, st);
   MISA_TC_CASE(16, 1)
   MISA_TC_CASE(32, 1)
   MISA_TC_CASE(48, 1)

@@ -46,7 +46,10 @@ def test_workspace_sizes(lib):
     assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 16) + hp(32)
     assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 64) + hp(32)
     assert ws(2, 1, 16, 64, 128, 2048, 64, 8, 256, 512) == 256 + 16 * 2048 * 4 + tc(16, 16)
-    assert ws(4, 16, 1, 64, 128, 131072, 64, 8, 2048, 8192) == 256 + 2 * 16 * 8192 * 4 + 256
+    # re-rank: sorted candidate ids, their scores, per-row counts, tensor-core scratch
+    # (every row in the decode form with all 64 heads)
+    assert ws(4, 16, 1, 64, 128, 131072, 64, 8, 2048, 8192) == \
+        256 + 2 * 16 * 8192 * 4 + 256 + tc(16, 64)
     # invalid sizes report 0
     assert ws(1, 0, 1, 64, 128, 1024, 64, 8, 16, 16) == 0
     assert ws(1, 1, 1, 64, 128, 1024, 64, 65, 16, 16) == 0

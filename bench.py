@@ -285,6 +285,14 @@ def run_cuda(args, wl):
         q, w, k, pos = sets[i % 2]
         M.dsa_score_topk(q, w, k, pos, wl.topk, idx=didx, vals=dvals)
 
+    def kept_pool_step(i):
+        # decode with the pooled keys kept between steps: each sequence's newest key (the
+        # query's own position, L - 1) is the only change, so only its block is re-pooled
+        q, w, k, pos = sets[i % 2]
+        M.misa_pool_keys_range(k, wl.B, kp[i % 2], wl.L - 1, wl.L)
+        M.misa_route_heads(q, w, k, kp[i % 2], pos, wl.B, wl.h, heads=heads)
+        M.misa_score_topk(q, w, k, heads, pos, wl.topk, idx=idx, vals=vals)
+
     def barrier():
         if world > 1:
             dist.barrier()
@@ -326,6 +334,8 @@ def run_cuda(args, wl):
     score_ms_avg = call_ms[2]
     ms_dagger = timed(dagger_step, args.steps, args.warmup)
     ms_dsa = timed(dsa_step, args.steps, args.warmup)
+    decode = T == 1 and bool(np.all(x.pos == wl.L - 1))
+    ms_kept = timed(kept_pool_step, args.steps, args.warmup) if decode else None
     # the routed scoring kernel alone (misa_score_rows: the scorer of misa_score_topk with the
     # same launch configuration), on the heads the MISA steps routed
     score_buf = torch.empty((nseq, T, wl.L), dtype=torch.float32, device=dev)
@@ -376,6 +386,10 @@ def run_cuda(args, wl):
                     "algorithmic_bytes": score_bytes, "avg_ms": ms_score_kernel}
 
     launches_per_step = misa_step_launches(wl)
+    if ms_kept is not None:
+        kept = {"value": units * world / (ms_kept * 1e-3), "ms_per_step": ms_kept,
+                "speedup_vs_dsa": ms_dsa / ms_kept,
+                "step": "refresh the newest key's pooled block + route + routed score + top-k"}
     line = {
         "metric": METRIC, "value": units * world / (ms_misa * 1e-3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_misa,
@@ -402,6 +416,8 @@ def run_cuda(args, wl):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if ms_kept is not None:
+        line["paths"]["misa_kept_pool"] = kept
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

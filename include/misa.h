@@ -95,6 +95,19 @@ int misa_pool_keys(const uint16_t* k, int nseq, int64_t L, int d, int B, float* 
                    void* stream);
 
 /*
+ * Refresh of the pooled keys after keys changed: recomputes, for every sequence,
+ * exactly the blocks of Eq. (4) that meet the token range [s_begin, s_end) and
+ * leaves every other block of k_pool as it is.  The pages count the router as
+ * O(H * M) per query, which presumes the pooled keys are kept rather than rebuilt;
+ * in decode a step appends one key, so the caller refreshes [pos, pos + 1) and only
+ * that key's block is re-read (B keys instead of L).  Same layout as
+ * misa_pool_keys; 0 <= s_begin <= s_end <= L, else MISA_ERR_INVALID_ARG; an empty
+ * range launches nothing.  No workspace.
+ */
+int misa_pool_keys_range(const uint16_t* k, int nseq, int64_t L, int d, int B,
+                         int64_t s_begin, int64_t s_end, float* k_pool, void* stream);
+
+/*
  * Block-pooled head router, Eqs. (7)-(8) (Methodology section 1).  For query
  * (n, t) with prefix P = pos+1 and M = ceil(P/B) blocks of that prefix:
  *   A[j, b] = w[j] * ReLU(q[j] . kp_b),   E[j] = (1/M) * sum_b |A[j, b]|,
@@ -146,10 +159,11 @@ int misa_score_rows(const uint16_t* q, const float* w, const uint16_t* k, const 
 
 /*
  * MISA-dagger fine stage, Eq. (12) (Methodology section 2): for each query,
- * re-score the candidate tokens cand[n, t, 0 .. kprime-1] (int32, distinct ids;
- * -1 = empty slot) with all H heads, I[s] = sum_j w[j] * ReLU(q[j] . k[s]), and
- * return the topk best (ties: lower token index).  Candidates outside
- * [0, pos] are recorded as bad device input and skipped.
+ * re-score the candidate tokens cand[n, t, 0 .. kprime-1] (int32, any order;
+ * -1 = empty slot; a repeated id counts once) with all H heads,
+ * I[s] = sum_j w[j] * ReLU(q[j] . k[s]), and return the topk best (ties: lower
+ * token index).  Candidates outside [0, pos] are recorded as bad device input and
+ * skipped.
  * Needs misa_workspace_size(MISA_OP_DAGGER_RERANK, ...).
  */
 int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k,

@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     misa_check_device_status,
     misa_dagger_rerank,
     misa_pool_keys,
+    misa_pool_keys_range,
     misa_route_heads,
     misa_score_rows,
     misa_score_topk,

@@ -33,6 +33,8 @@ _SIGS = {
     "misa_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int,
                                     _c_int, _c_int, _c_int]),
     "misa_pool_keys": (_c_int, [_p, _c_int, _c_i64, _c_int, _c_int, _p, _p]),
+    "misa_pool_keys_range": (_c_int, [_p, _c_int, _c_i64, _c_int, _c_int, _c_i64, _c_i64, _p,
+                                      _p]),
     "misa_route_heads": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_i64,
                                   _c_int, _c_int, _p, _p, _p, _c_sz, _p]),
     "misa_score_topk": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int, _c_i64,
@@ -150,6 +152,21 @@ def misa_pool_keys(k: torch.Tensor, B: int, out: torch.Tensor | None = None) -> 
     _check("misa_pool_keys",
            _lib.misa_pool_keys(_ptr(k), nseq, L, d, B, _ptr(out), _stream()))
     return out
+
+
+def misa_pool_keys_range(k: torch.Tensor, B: int, k_pool: torch.Tensor, s_begin: int,
+                         s_end: int) -> torch.Tensor:
+    """Recompute, in place, the pooled blocks of k_pool that meet tokens [s_begin, s_end)
+    of every sequence (the keys there changed); other blocks are left as they are."""
+    k = _bits(k, "k")
+    nseq, L, d = k.shape
+    k_pool = _dev(k_pool, "k_pool", torch.float32)
+    if tuple(k_pool.shape) != (nseq, -(-L // B), d):
+        raise ValueError(f"k_pool must be [{nseq}, {-(-L // B)}, {d}], got {tuple(k_pool.shape)}")
+    _check("misa_pool_keys_range",
+           _lib.misa_pool_keys_range(_ptr(k), nseq, L, d, B, int(s_begin), int(s_end),
+                                     _ptr(k_pool), _stream()))
+    return k_pool
 
 
 def misa_route_heads(q, w, k, k_pool, pos, B: int, h: int, return_E: bool = False,

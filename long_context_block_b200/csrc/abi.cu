@@ -155,6 +155,18 @@ int misa_pool_keys(const uint16_t* k, int nseq, int64_t L, int d, int B, float* 
   return cuda_status(launch_pool_mean(k, nseq, L, B, k_pool, (cudaStream_t)stream));
 }
 
+int misa_pool_keys_range(const uint16_t* k, int nseq, int64_t L, int d, int B,
+                         int64_t s_begin, int64_t s_end, float* k_pool, void* stream) {
+  MISA_TRY(check_shape(nseq, 1, 1, d, L));
+  if (B < 1 || s_begin < 0 || s_end < s_begin || s_end > L) return MISA_ERR_INVALID_ARG;
+  const int64_t M = (L + B - 1) / B;
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(k_pool, (size_t)nseq * M * d * 4, 16));
+  if (s_end == s_begin) return MISA_OK;
+  return cuda_status(
+      launch_pool_mean(k, nseq, L, B, k_pool, (cudaStream_t)stream, s_begin, s_end));
+}
+
 int misa_route_heads(const uint16_t* q, const float* w, const uint16_t* k, const float* k_pool,
                      const int32_t* pos, int nseq, int T, int H, int d, int64_t L, int B, int h,
                      int32_t* heads, float* E, void* ws, size_t ws_bytes, void* stream) {

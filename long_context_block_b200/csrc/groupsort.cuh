@@ -101,3 +101,158 @@ __device__ bool group_sort_desc(const uint64_t* in, uint32_t cnt, uint64_t* out,
 }
 
 }  // namespace misa
+
+namespace misa {
+
+// Bytes of shared memory group_sort_adaptive needs besides its bucket array: a word per
+// histogram bin (candidate counts, then bucket offsets) and a byte per bin (sub-bucket
+// bits).
+constexpr int kAdaptiveAuxBytes = kScoreHistBins * 4 + kScoreHistBins;
+
+// Descending sort like group_sort_desc, for candidates whose keys spread over many bins
+// unevenly (rows whose cutoff reaches far down, or short rows taken whole): bin b of
+// [blo, bhi] gets 2^s_b sub-buckets on the key bits below the bin, s_b chosen from the
+// bin's own candidate count (about two pairs per sub-bucket) and lowered uniformly until
+// the sub-buckets fit kSubBuckets.  `aux`: kAdaptiveAuxBytes of shared memory.  Same
+// contract and fallback signal as group_sort_desc.
+template <int NT>
+__device__ bool group_sort_adaptive(const uint64_t* in, uint32_t cnt, uint64_t* out,
+                                    uint32_t* buckets, uint8_t* aux, uint32_t blo, uint32_t bhi,
+                                    uint32_t* warp_sums, uint32_t& s_flag, uint32_t& s_tot) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  constexpr int kWarps = NT / 32;
+  constexpr int kPerB = kScoreHistBins / NT;   // bins per thread, highest bins first
+  uint32_t* binw = reinterpret_cast<uint32_t*>(aux);   // counts, then bucket offsets
+  uint8_t* bshift = aux + kScoreHistBins * 4;
+  const uint32_t nb = bhi - blo + 1;
+  for (uint32_t i = t; i < nb; i += NT) binw[i] = 0;
+  if (t == 0) s_flag = 0;
+  __syncthreads();
+  for (uint32_t i = t; i < cnt; i += NT)
+    atomicAdd(&binw[(uint32_t)(in[i] >> (64 - kScoreHistBits)) - blo], 1u);
+  __syncthreads();
+  // desired sub-bucket bits per bin: 2^s >= count / 2
+  int s0[kPerB];
+#pragma unroll
+  for (int j = 0; j < kPerB; ++j) {
+    const uint32_t p = t * kPerB + j;   // position in descending bin order
+    const uint32_t c = p < nb ? binw[bhi - blo - p] : 0u;
+    const int lg = c <= 2 ? 0 : 32 - __clz(c - 1);   // ceil(log2 c)
+    s0[j] = min(max(lg - 1, 0), 32 - kScoreHistBits);
+  }
+  int delta = 0;
+  for (;; ++delta) {
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < kPerB; ++j)
+      if ((uint32_t)(t * kPerB + j) < nb) local += 1u << max(s0[j] - delta, 0);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+    if (lane == 0) warp_sums[warp] = local;
+    __syncthreads();
+    uint32_t tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) tot += warp_sums[w];
+    __syncthreads();
+    if (tot <= (uint32_t)kSubBuckets) break;   // nb <= kSubBuckets: ends by delta = 20
+  }
+  // bucket offsets in descending bin order
+  uint32_t sz[kPerB], local = 0;
+#pragma unroll
+  for (int j = 0; j < kPerB; ++j) {
+    const bool in_range = (uint32_t)(t * kPerB + j) < nb;
+    s0[j] = max(s0[j] - delta, 0);
+    sz[j] = in_range ? 1u << s0[j] : 0u;
+    local += sz[j];
+  }
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t run = incl - local, total = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t x = warp_sums[w];
+    if (w < warp) run += x;
+    total += x;
+  }
+  if (t == 0) s_tot = total;
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPerB; ++j) {
+    const uint32_t p = t * kPerB + j;
+    if (p < nb) {
+      binw[bhi - blo - p] = run;
+      bshift[bhi - blo - p] = (uint8_t)s0[j];
+    }
+    run += sz[j];
+  }
+  __syncthreads();
+  const uint32_t nsub = s_tot;
+  auto bucket_of = [&](uint64_t v) -> uint32_t {
+    const uint32_t key = (uint32_t)(v >> 32);
+    const uint32_t b = (key >> (32 - kScoreHistBits)) - blo;
+    const uint32_t s = bshift[b];
+    const uint32_t sub = s ? (key >> (32 - kScoreHistBits - s)) & ((1u << s) - 1u) : 0u;
+    return binw[b] + ((1u << s) - 1u - sub);   // larger keys -> smaller bucket numbers
+  };
+  for (uint32_t i = t; i < nsub; i += NT) buckets[bpad(i)] = 0;
+  __syncthreads();
+  for (uint32_t i = t; i < cnt; i += NT) atomicAdd(&buckets[bpad(bucket_of(in[i]))], 1u);
+  __syncthreads();
+  constexpr int kPer = kSubBuckets / NT;
+  uint32_t c[kPer], lsum = 0, big = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const uint32_t b = t * kPer + i;
+    c[i] = b < nsub ? buckets[bpad(b)] : 0u;
+    lsum += c[i];
+    big |= c[i] > kMaxBucket;
+  }
+  incl = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  if (big) s_flag = 1;
+  __syncthreads();
+  uint32_t r2 = 0;
+  for (int w = 0; w < warp; ++w) r2 += warp_sums[w];
+  r2 += incl - lsum;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const uint32_t b = t * kPer + i;
+    if (b < nsub) buckets[bpad(b)] = r2;
+    r2 += c[i];
+  }
+  __syncthreads();
+  if (s_flag) return false;
+  for (uint32_t i = t; i < cnt; i += NT) {
+    const uint64_t v = in[i];
+    out[atomicAdd(&buckets[bpad(bucket_of(v))], 1u)] = v;
+  }
+  __syncthreads();
+  for (uint32_t b = t; b < nsub; b += NT) {
+    const uint32_t e = buckets[bpad(b)];
+    const uint32_t s = b ? buckets[bpad(b - 1)] : 0u;
+    for (uint32_t i = s + 1; i < e; ++i) {
+      const uint64_t v = out[i];
+      uint32_t j = i;
+      while (j > s && out[j - 1] < v) {
+        out[j] = out[j - 1];
+        --j;
+      }
+      out[j] = v;
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+}  // namespace misa

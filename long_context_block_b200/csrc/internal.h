@@ -23,9 +23,10 @@ constexpr int kTopkCandCap = 16384;
 // Router: blocks of the prefix handled by one CTA of the partial-energy pass.
 constexpr int kRouteChunk = 32;
 
-// K1 -- mean pooling (pool.cu)
+// K1 -- mean pooling (pool.cu): every block, or only the blocks that meet the token range
+// [s_begin, s_end) (s_end < 0: up to L).
 cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, float* k_pool,
-                             cudaStream_t st);
+                             cudaStream_t st, int64_t s_begin = 0, int64_t s_end = -1);
 
 // K2 -- router: partial head energies per chunk of blocks, then E and top-h by the
 // last CTA of each row (route.cu).  `counters` is rows ints of scratch (zeroed here).

@@ -7,6 +7,9 @@
 // (8 dims) of the 256-byte key row, so every warp-wide load covers two whole rows
 // (512 contiguous bytes).  Eight token pairs are loaded before any is accumulated to
 // keep enough bytes in flight per SM.
+//
+// The same kernel refreshes a range of blocks: in decode a sequence gains one key per
+// step, so only the block holding it changes and the rest of the pooled keys are reused.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,18 +23,19 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4& v) {
   a[6] += bf16lo(v.w); a[7] += bf16hi(v.w);
 }
 
+// Blocks b0 .. b0 + Mu - 1 of every sequence (M blocks per sequence in `out`).
 __global__ void __launch_bounds__(256) pool_mean_kernel(const uint4* __restrict__ k, int nseq,
-                                                        int64_t L, int B, int M,
+                                                        int64_t L, int B, int M, int b0, int Mu,
                                                         float* __restrict__ out) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int half = lane >> 4;   // 0: even tokens of the block, 1: odd tokens
   const int vec = lane & 15;    // which 16-byte slice of the key row
-  const int64_t items = (int64_t)nseq * M;
+  const int64_t items = (int64_t)nseq * Mu;
   for (int64_t it = warp; it < items; it += nwarps) {
-    const int64_t n = it / M;
-    const int64_t b = it - n * M;
+    const int64_t n = it / Mu;
+    const int64_t b = b0 + (it - n * Mu);
     const int64_t s0 = b * B;
     const int64_t s1 = min(s0 + (int64_t)B, L);
     const uint4* base = k + n * L * 16 + vec;   // a key row is 16 uint4
@@ -49,7 +53,7 @@ __global__ void __launch_bounds__(256) pool_mean_kernel(const uint4* __restrict_
     for (int i = 0; i < 8; ++i) a[i] += __shfl_down_sync(0xffffffffu, a[i], 16);
     if (half == 0) {
       const float inv = 1.0f / (float)(s1 - s0);
-      float4* o = reinterpret_cast<float4*>(out + it * kHeadDim + vec * 8);
+      float4* o = reinterpret_cast<float4*>(out + (n * M + b) * kHeadDim + vec * 8);
       o[0] = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
       o[1] = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
     }
@@ -59,15 +63,19 @@ __global__ void __launch_bounds__(256) pool_mean_kernel(const uint4* __restrict_
 }  // namespace
 
 cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, float* k_pool,
-                             cudaStream_t st) {
+                             cudaStream_t st, int64_t s_begin, int64_t s_end) {
   const int M = (int)((L + B - 1) / B);
-  const int64_t items = (int64_t)nseq * M;
+  if (s_end < 0) s_end = L;
+  const int b0 = (int)(s_begin / B);
+  const int Mu = (int)((s_end + B - 1) / B) - b0;   // blocks meeting [s_begin, s_end)
+  if (Mu <= 0) return cudaSuccess;
+  const int64_t items = (int64_t)nseq * Mu;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (items + 7) / 8;           // 8 warps per CTA
   const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  pool_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M,
+  pool_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M, b0, Mu,
                                          k_pool);
   return cudaGetLastError();
 }

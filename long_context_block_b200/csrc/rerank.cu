@@ -1,9 +1,14 @@
 // K7 (preparation): MISA-dagger candidate lists -- Eq. (12) of the MISA paper summary
 // (Methodology section 2) re-scores the coarse candidates Omega_t with all heads and
 // keeps the top k.  To make that final TopK resolve equal scores by token index with
-// the ordinary index-order pass, each row's candidates are first sorted ascending.
-// Empty slots (-1) and ids outside the query's prefix are dropped (the latter are
+// the ordinary index-order pass, each row's candidates are first put in ascending token
+// order.  Empty slots (-1) and ids outside the query's prefix are dropped (the latter are
 // recorded as bad device input); `count` receives the number of valid candidates.
+//
+// Omega_t is a set of token ids inside the prefix [0, P), so the ordering is a bitmap
+// compaction: one bit per prefix token in shared memory, set by the candidates, then a
+// block-wide scan of the words' popcounts writes the ids in ascending order (a repeated
+// id counts once).  Prefixes too long for a shared-memory bitmap take a bitonic sort.
 #include "blocksort.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -12,6 +17,60 @@ namespace misa {
 namespace {
 
 constexpr int kThreads = kSortThreads;
+constexpr int kBitmapThreads = 512;
+constexpr int kBitmapMaxBytes = 200 * 1024;
+
+__global__ void __launch_bounds__(kBitmapThreads) bitmap_candidates_kernel(
+    const int32_t* __restrict__ cand, const int32_t* __restrict__ pos, int64_t L, int kprime,
+    int32_t* __restrict__ sorted, int32_t* __restrict__ count, int* status, int64_t row0) {
+  extern __shared__ uint32_t bm[];   // [ceil(P / 32)] words
+  __shared__ uint32_t warp_sums[kBitmapThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t row = row0 + blockIdx.x;
+  const int P = prefix_len(pos, row, L, tid == 0 ? status : nullptr);
+  const int nwords = (P + 31) >> 5;
+  for (int i = tid; i < nwords; i += kBitmapThreads) bm[i] = 0u;
+  __syncthreads();
+  const int32_t* c_row = cand + row * kprime;
+  for (int i = tid; i < kprime; i += kBitmapThreads) {
+    const int32_t c = c_row[i];
+    if (c >= 0 && c < P)
+      atomicOr(&bm[c >> 5], 1u << (c & 31));
+    else if (c != -1)
+      set_status(status, MISA_ERR_BAD_DEVICE_INPUT);
+  }
+  __syncthreads();
+  // thread t owns words [t * per, (t + 1) * per)
+  const int per = (nwords + kBitmapThreads - 1) / kBitmapThreads;
+  const int w0 = min(tid * per, nwords), w1 = min(w0 + per, nwords);
+  uint32_t local = 0;
+  for (int i = w0; i < w1; ++i) local += __popc(bm[i]);
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t off = incl - local, total = 0;
+  for (int w = 0; w < kBitmapThreads / 32; ++w) {
+    const uint32_t s = warp_sums[w];
+    if (w < warp) off += s;
+    total += s;
+  }
+  int32_t* out = sorted + row * kprime;
+  for (int i = w0; i < w1; ++i) {
+    uint32_t b = bm[i];
+    while (b) {
+      const int bit = __ffs(b) - 1;
+      out[off++] = i * 32 + bit;
+      b &= b - 1u;
+    }
+  }
+  for (int i = (int)total + tid; i < kprime; i += kBitmapThreads) out[i] = -1;
+  if (tid == 0) count[row] = (int32_t)total;
+}
 
 __global__ void __launch_bounds__(kThreads) sort_candidates_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pos, int64_t L, int kprime,
@@ -53,15 +112,25 @@ __global__ void __launch_bounds__(kThreads) sort_candidates_kernel(
 cudaError_t launch_sort_candidates(const int32_t* cand, const int32_t* pos, int rows,
                                    int64_t L, int kprime, int32_t* sorted, int32_t* count,
                                    int* status, cudaStream_t st) {
+  const size_t bm_bytes = (size_t)((L + 31) / 32) * sizeof(uint32_t);
+  const bool bitmap = bm_bytes <= (size_t)kBitmapMaxBytes;
   const int sortn = topk_sort_size(kprime);
-  const size_t smem = (size_t)sortn * sizeof(uint64_t);
-  cudaError_t e = cudaFuncSetAttribute(sort_candidates_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = bitmap ? bm_bytes : (size_t)sortn * sizeof(uint64_t);
+  cudaError_t e = bitmap ? cudaFuncSetAttribute(bitmap_candidates_kernel,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem)
+                         : cudaFuncSetAttribute(sort_candidates_kernel,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem);
   if (e != cudaSuccess) return e;
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
-    sort_candidates_kernel<<<(unsigned)nr, kThreads, smem, st>>>(cand, pos, L, kprime, sortn,
-                                                                 sorted, count, status, row0);
+    if (bitmap)
+      bitmap_candidates_kernel<<<(unsigned)nr, kBitmapThreads, smem, st>>>(
+          cand, pos, L, kprime, sorted, count, status, row0);
+    else
+      sort_candidates_kernel<<<(unsigned)nr, kThreads, smem, st>>>(cand, pos, L, kprime, sortn,
+                                                                   sorted, count, status, row0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

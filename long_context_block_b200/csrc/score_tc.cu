@@ -42,6 +42,7 @@ constexpr int kKeyTileBytes = kTileKeys * kHeadDim * 2;   // 32 KB
 constexpr int kKeyHalfBytes = kKeyTileBytes / 2;           // [128 rows][64 cols] bf16
 constexpr long long kWaitCycles = 4000000000LL;            // ~2 s at the top SM clock
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kIdAhead = 4;                                 // gather ids loaded ahead (tiles)
 
 template <int HS, int QB>
 struct Cfg {
@@ -137,7 +138,8 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     const float* __restrict__ wsel, const int32_t* __restrict__ pos,
     const int32_t* __restrict__ tile_off, int units, Units geo, int64_t L,
     float* __restrict__ out, int64_t out_stride, int* status, uint32_t* __restrict__ hist,
-    const int32_t* __restrict__ gidx, const int32_t* __restrict__ glen) {
+    const int32_t* __restrict__ gidx, const int32_t* __restrict__ glen,
+    const uint16_t* __restrict__ kraw) {
   using C = Cfg<HS, QB>;
   constexpr int N = C::N;
   constexpr int kEpiThreads = 32 * C::kEpiWarps;
@@ -168,7 +170,11 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     for (int b = tid; b < kScoreHistBins; b += C::kThreads) shist[b] = 0;
 
   if (tid == 0) {
-    for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    // a gathered tile completes with one cp.async arrival per producer lane
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], gidx ? 32 : 1);
+      mbar_init(&empty[s], 1);
+    }
     for (int s = 0; s < C::kQBufs; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
     for (int s = 0; s < C::kWBufs; ++s) {
       mbar_init(&wfull[s], 1);
@@ -223,20 +229,36 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
       ++qissued;
       ++wissued;
       const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
-      // gather mode (QB == 1, unit = row): the row's token list and its length
+      // gather mode (QB == 1, unit = row): the row's token list and its length; lane l
+      // gathers keys 4l .. 4l+3 of a tile, whose ids it loads kIdAhead tiles early
       const int32_t* ids = gidx ? gidx + (int64_t)sg.u * out_stride : nullptr;
       const int cnt = gidx ? min(max(glen[sg.u], 0), (int)out_stride) : 0;
+      int32_t rq[kIdAhead][4];
+      auto fetch_ids = [&](int jj, int32_t(&r)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = jj * kTileKeys + 4 * lane + i;
+          int32_t id = c < cnt ? ids[c] : 0;   // padding keys are masked by the epilogue
+          if (id < 0 || id >= L) id = 0;
+          r[i] = (int32_t)(y0 + id);
+        }
+      };
+      if (ids) {
+#pragma unroll
+        for (int d = 0; d < kIdAhead; ++d)
+          if (sg.a + d < sg.b) fetch_ids(sg.a + d, rq[d]);
+      }
       for (int j = sg.a; j < sg.b; ++j) {
         const int s = issued % C::kStages;
         int32_t r[4];
-        if (ids) {   // fetch the ids before the wait so their latency hides behind it
+        if (ids) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = j * kTileKeys + 4 * lane + i;
-            int32_t id = c < cnt ? ids[c] : 0;   // padding keys are masked by the epilogue
-            if (id < 0 || id >= L) id = 0;
-            r[i] = (int32_t)(y0 + id);
-          }
+          for (int i = 0; i < 4; ++i) r[i] = rq[0][i];
+#pragma unroll
+          for (int d = 0; d + 1 < kIdAhead; ++d)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rq[d][i] = rq[d + 1][i];
+          if (j + kIdAhead < sg.b) fetch_ids(j + kIdAhead, rq[kIdAhead - 1]);
         }
         if (!warp_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status)) {
           ok = false;
@@ -244,11 +266,20 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
         }
         uint8_t* kb = base + C::kStageBase + s * kKeyTileBytes;
         if (ids) {
-          if (lane == 0) mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
-          __syncwarp();
-          uint8_t* dst = kb + lane * 4 * 128;   // rows 4*lane .. 4*lane+3 of both halves
-          tma_gather4(dst, &tm_k, &full[s], 0, r[0], r[1], r[2], r[3]);
-          tma_gather4(dst + kKeyHalfBytes, &tm_k, &full[s], 64, r[0], r[1], r[2], r[3]);
+          // 64 warp-wide steps, two key rows each: lanes 0-15 copy row 2i, lanes 16-31 row
+          // 2i+1, 16 bytes per lane, into the 128-byte-swizzled halves of the tile.  Row
+          // 4m+e's id sits in lane m's r[e].
+          const int c = lane & 15, odd = lane >> 4;
+          const uint32_t kb_s = smem_u32(kb) + (uint32_t)((c >> 3) * kKeyHalfBytes);
+#pragma unroll
+          for (int i = 0; i < kTileKeys / 2; ++i) {
+            const int32_t ya = __shfl_sync(0xffffffffu, r[2 * (i & 1)], i >> 1);
+            const int32_t yb = __shfl_sync(0xffffffffu, r[2 * (i & 1) + 1], i >> 1);
+            const int row = 2 * i + odd;
+            const uint32_t dst = kb_s + (uint32_t)(row * 128) + (uint32_t)(((c & 7) ^ (row & 7)) << 4);
+            cp_async16(dst, kraw + (int64_t)(odd ? yb : ya) * kHeadDim + c * 8);
+          }
+          cp_async_mbar_arrive(&full[s]);
         } else if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
           const int32_t y = (int32_t)(y0 + (int64_t)j * kTileKeys);
@@ -291,6 +322,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
             break;
           }
           tc_fence_after();
+          if (gidx) fence_proxy_async_smem();   // gathered tile was written by cp.async
           const uint32_t kaddr = smem0 + C::kStageBase + s * kKeyTileBytes;
           const uint32_t d = tmem_base + (uint32_t)(acc * C::kAccStride);
 #pragma unroll
@@ -521,7 +553,8 @@ template <int HS, int QB>
 cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float* wg,
                        const int32_t* pos, const int32_t* tile_off, int units, Units geo,
                        int64_t L, float* out, int64_t out_stride, int* status, uint32_t* hist,
-                       const int32_t* gidx, const int32_t* glen, cudaStream_t st) {
+                       const int32_t* gidx, const int32_t* glen, const uint16_t* kraw,
+                       cudaStream_t st) {
   using C = Cfg<HS, QB>;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -530,7 +563,7 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   score_tc_kernel<HS, QB><<<sms, C::kThreads, C::kSmemBytes, st>>>(
-      tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist, gidx, glen);
+      tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist, gidx, glen, kraw);
   return cudaGetLastError();
 }
 
@@ -600,15 +633,14 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
                                                glen, (int)out_stride, qg, wg, tile_off, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // key rows come as whole 128-key tiles, or one row per box for the gather
-  CUtensorMap tk, tq;
-  if (!make_map(&tk, k, (uint64_t)nseq * L, gather ? 1u : (uint32_t)kTileKeys) ||
+  CUtensorMap tk, tq;   // (the gather copies key rows with cp.async: tk goes unused)
+  if (!make_map(&tk, k, (uint64_t)nseq * L, (uint32_t)kTileKeys) ||
       !make_map(&tq, qg, (uint64_t)units * p.N, (uint32_t)p.N))
     return cudaErrorInvalidValue;
 #define MISA_TC_CASE(HS_, QB_)                                                                  \
   if (p.HS == HS_ && p.QB == QB_)                                                               \
     return launch_cfg<HS_, QB_>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, \
-                                hist, gidx, glen, st);
+                                hist, gidx, glen, k, st);
   MISA_TC_CASE(16, 1)
   MISA_TC_CASE(32, 1)
   MISA_TC_CASE(48, 1)

@@ -606,15 +606,33 @@ __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
 }
 
 // ---------------------------------------------------------------- row-resident form
-// Rows of up to kRowCap scores and k <= kRowCandCap: one CTA of kSelThreads threads per
-// row keeps the row's keys in shared memory, finds the cutoff bin with a shared-memory
-// histogram of the top kScoreHistBits key bits, compacts the candidates (bins at or above
-// it) and sorts them with the counting sort.  A crowded cutoff falls back to an exact
-// radix select over the resident keys.
+// Rows of up to kRowCap scores and k <= CAP: one CTA of NT threads per row keeps the row's
+// keys in shared memory, finds the cutoff bin with a shared-memory histogram of the top
+// kScoreHistBits key bits, compacts the candidates (bins at or above it) and sorts them
+// with the counting sort.  A crowded cutoff (more than CAP candidates) takes an exact
+// radix select over the resident keys instead.  Three shapes: 256 threads and 3072
+// candidates (two CTAs per SM, many rows, k <= 3072), 512 or 1024 threads and 8192
+// candidates (one CTA per SM; 1024 threads when there are too few rows to fill the SMs).
 constexpr int kRowCap = 16384;
-constexpr int kRowCandCap = 3072;   // keeps two CTAs per SM
 constexpr int kRowLoadUnroll = 8;
 
+template <int NT, int CAP>
+struct RowCfg {
+  // keys [kRowCap] u32, later the sorted pairs [<= CAP] u64, then the candidates [CAP] u64
+  static constexpr int kKeyPairs = kRowCap / 2 > CAP ? kRowCap / 2 : CAP;
+  // the adaptive sort's bin tables sit in the key space the sorted pairs leave free, or
+  // after the candidates
+  static constexpr bool kAuxInKeys = (kKeyPairs - CAP) * 8 >= kAdaptiveAuxBytes;
+  static constexpr size_t kAuxOff = kAuxInKeys ? (size_t)CAP * 8 : (size_t)(kKeyPairs + CAP) * 8;
+  static constexpr size_t kSmem =
+      (size_t)(kKeyPairs + CAP) * sizeof(uint64_t) + (kAuxInKeys ? 0 : kAdaptiveAuxBytes);
+  static constexpr int kEMax = CAP <= NT ? 1 : CAP <= 2 * NT ? 2 : CAP <= 4 * NT ? 4
+                               : CAP <= 8 * NT ? 8 : 16;
+  static constexpr int kBinsPer = 2048 / NT;   // radix-select bins per thread
+  static_assert(CAP <= 16 * NT && 2048 % NT == 0, "row kernel shape");
+};
+
+template <int NT>
 __device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_t* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -630,63 +648,82 @@ __device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_
   hi = red[1];
 }
 
-__global__ void __launch_bounds__(kSelThreads, 2) topk_row_kernel(
+// Bitonic fallback of the counting sort: sorted[0 .. sortn) descending, sortn = NT * 2^i.
+template <int NT, int EMAX>
+__device__ __forceinline__ void row_bitonic(uint64_t* sorted, int sortn) {
+  const int e = sortn / NT;
+  if (e <= 1) sort_buf_desc_e<1, NT>(sorted);
+  else if constexpr (EMAX >= 2) {
+    if (e == 2) sort_buf_desc_e<2, NT>(sorted);
+    else if constexpr (EMAX >= 4) {
+      if (e == 4) sort_buf_desc_e<4, NT>(sorted);
+      else if constexpr (EMAX >= 8) {
+        if (e == 8) sort_buf_desc_e<8, NT>(sorted);
+        else if constexpr (EMAX >= 16) sort_buf_desc_e<16, NT>(sorted);
+      }
+    }
+  }
+}
+
+template <int NT, int CAP, int MINB>
+__global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
     int32_t* __restrict__ idx, float* __restrict__ vals, int64_t row0) {
+  using RC = RowCfg<NT, CAP>;
   extern __shared__ uint64_t rbuf[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(rbuf);          // [kRowCap] keys, then
-  uint64_t* sorted = rbuf;                                     //   [kRowCandCap] sorted pairs
-  uint64_t* cand = rbuf + kRowCap / 2;                         // [kRowCandCap] candidates
+  uint64_t* sorted = rbuf;                                     //   [CAP] sorted pairs
+  uint64_t* cand = rbuf + RC::kKeyPairs;                       // [CAP] candidates
   __shared__ __align__(16) uint32_t hist[kSubBucketWords];     // histogram, then buckets
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t red[2];
-  __shared__ uint32_t s_cut, s_total, s_big, s_fill, s_flag, s_digit, s_above, s_top;
-  const int t = threadIdx.x, lane = t & 31;
+  __shared__ uint32_t s_cut, s_total, s_big, s_fill, s_flag, s_digit, s_above, s_top, s_nsub;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t row = row0 + blockIdx.x;
   const int n = gather_len ? gather_len[row] : prefix_len(pos, row, L, nullptr);
   const uint32_t target = (uint32_t)min(n, topk);
   const float* x = scores + row * stride;
   const int32_t* imap = index_map ? index_map + row * stride : nullptr;
 
-  for (int b = t; b < kScoreHistBins; b += kSelThreads) hist[b] = 0;
+  for (int b = t; b < kScoreHistBins; b += NT) hist[b] = 0;
   if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; s_fill = 0; s_top = 0; }
-  for (int base = 0; base < n; base += kSelThreads * kRowLoadUnroll) {
+  for (int base = 0; base < n; base += NT * kRowLoadUnroll) {
     float v[kRowLoadUnroll];
 #pragma unroll
     for (int j = 0; j < kRowLoadUnroll; ++j) {
-      const int e = base + j * kSelThreads + t;
+      const int e = base + j * NT + t;
       v[j] = e < n ? x[e] : 0.f;
     }
 #pragma unroll
     for (int j = 0; j < kRowLoadUnroll; ++j) {
-      const int e = base + j * kSelThreads + t;
+      const int e = base + j * NT + t;
       if (e < n) keys[e] = score_key(v[j]);
     }
   }
   __syncthreads();
   uint32_t cut, btop, C;
-  if ((uint32_t)n <= (uint32_t)kRowCandCap) {
-    // every score is a candidate
+  if ((uint32_t)n <= target) {
+    // every score is selected
     uint32_t lo = 0xffffffffu, hi = 0;
-    for (int e = t; e < n; e += kSelThreads) {
+    for (int e = t; e < n; e += NT) {
       const uint32_t b = keys[e] >> (32 - kScoreHistBits);
       lo = min(lo, b);
       hi = max(hi, b);
     }
-    block_minmax(lo, hi, red);
+    block_minmax<NT>(lo, hi, red);
     cut = lo;
     btop = hi;
     C = (uint32_t)n;
   } else {
-    for (int e = t; e < n; e += kSelThreads) atomicAdd(&hist[keys[e] >> (32 - kScoreHistBits)], 1u);
+    for (int e = t; e < n; e += NT) atomicAdd(&hist[keys[e] >> (32 - kScoreHistBits)], 1u);
     __syncthreads();
-    HistView<kSelThreads> hv;
-    cut = hist_cutoff<kSelThreads>(hist, target, hv, warp_sums, s_cut, s_total, s_big);
+    HistView<NT> hv;
+    cut = hist_cutoff<NT>(hist, target, hv, warp_sums, s_cut, s_total, s_big);
     // highest occupied bin
     uint32_t top = 0;
 #pragma unroll
-    for (int i = HistView<kSelThreads>::kPer - 1; i >= 0; --i)
+    for (int i = HistView<NT>::kPer - 1; i >= 0; --i)
       if (hv.c[i]) top = max(top, (uint32_t)(hv.hi - 1 - i));
     if (top) atomicMax(&s_top, top);
     __syncthreads();
@@ -694,9 +731,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_row_kernel(
     C = s_total;
   }
   __syncthreads();
-  const bool fits = C <= (uint32_t)kRowCandCap;
+  const bool fits = C <= (uint32_t)CAP;
   if (fits) {
-    for (int base = 0; base < n; base += kSelThreads) {
+    for (int base = 0; base < n; base += NT) {
       const int e = base + t;
       const uint32_t key = e < n ? keys[e] : 0u;
       const bool take = e < n && (key >> (32 - kScoreHistBits)) >= cut;
@@ -713,28 +750,28 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_row_kernel(
     for (int p = 0; p < 3; ++p) {
       const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
       const int nb = p == 2 ? 1024 : 2048;
-      for (int b = t; b < 2048; b += kSelThreads) hist[b] = 0;
+      for (int b = t; b < 2048; b += NT) hist[b] = 0;
       __syncthreads();
-      for (int e = t; e < n; e += kSelThreads) {
+      for (int e = t; e < n; e += NT) {
         const uint32_t key = keys[e];
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
       }
       __syncthreads();
-      // suffix scan: thread t covers bins nb-1-8t .. nb-8t (8 bins each)
-      uint32_t cb[8], local = 0;
+      // suffix scan: thread t covers bins nb-1-kBinsPer*t-i, i < kBinsPer
+      uint32_t cb[RC::kBinsPer], local = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int b = nb - 1 - 8 * t - i;
+      for (int i = 0; i < RC::kBinsPer; ++i) {
+        const int b = nb - 1 - RC::kBinsPer * t - i;
         cb[i] = b >= 0 ? hist[b] : 0u;
         local += cb[i];
       }
       uint32_t tot;
-      const uint32_t excl = block_excl_scan_nt<kSelThreads>(local, warp_sums, tot);
+      const uint32_t excl = block_excl_scan_nt<NT>(local, warp_sums, tot);
       uint32_t run = excl;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < RC::kBinsPer; ++i) {
         if (run < kneed && kneed <= run + cb[i]) {
-          s_digit = nb - 1 - 8 * t - i;
+          s_digit = nb - 1 - RC::kBinsPer * t - i;
           s_above = run;
         }
         run += cb[i];
@@ -746,49 +783,65 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_row_kernel(
       __syncthreads();
     }
     const uint32_t thr = prefix;
-    uint32_t eq_taken = 0;
-    for (int base = 0; base < n; base += kSelThreads) {
-      const int e = base + t;
-      const uint32_t key = e < n ? keys[e] : 0u;
-      const bool gt = e < n && key > thr;
-      const bool eq = e < n && key == thr;
-      uint32_t tot;
-      const uint32_t ex =
-          block_excl_scan_nt<kSelThreads>((gt ? 1u << 16 : 0u) | (eq ? 1u : 0u), warp_sums, tot);
-      const uint32_t re = eq_taken + (ex & 0xffffu);
-      const bool take = gt || (eq && re < kneed);
-      const uint32_t m = __ballot_sync(0xffffffffu, take);
-      uint32_t wb = 0;
-      if (lane == 0 && m) wb = atomicAdd(&s_fill, (uint32_t)__popc(m));
-      wb = __shfl_sync(0xffffffffu, wb, 0);
-      if (take) cand[wb + __popc(m & ((1u << lane) - 1u))] = compose(key, imap ? imap[e] : e);
-      eq_taken += tot & 0xffffu;
+    // Warp w compacts the contiguous slice [w0, w1) of the row in 32-key steps, so that
+    // ranks in (warp, step, lane) order are ranks in index order: one block scan places
+    // every warp's keys above the threshold and its equal ones.
+    constexpr int kWarps = NT / 32;
+    const int wper = (((n + kWarps - 1) / kWarps) + 31) & ~31;
+    const int w0 = min(warp * wper, n), w1 = min(w0 + wper, n);
+    uint32_t ngt = 0, neq = 0;
+    for (int e = w0 + lane; e < w1; e += 32) {
+      const uint32_t key = keys[e];
+      ngt += key > thr;
+      neq += key == thr;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+      neq += __shfl_xor_sync(0xffffffffu, neq, o);
+    }
+    uint32_t tot;   // n <= kRowCap < 2^16: both counts fit 16 bits
+    const uint32_t ex = block_excl_scan_nt<NT>(lane == 0 ? (ngt << 16) | neq : 0u, warp_sums, tot);
+    const uint32_t wex = __shfl_sync(0xffffffffu, ex, 0);
+    const uint32_t G = tot >> 16;   // keys above the threshold = target - kneed
+    uint32_t gpos = wex >> 16, epos = wex & 0xffffu;
+    for (int e0 = w0; e0 < w1; e0 += 32) {
+      const int e = e0 + lane;
+      const uint32_t key = e < w1 ? keys[e] : 0u;
+      const bool gt = e < w1 && key > thr;
+      const bool eq = e < w1 && key == thr;
+      const uint32_t mg = __ballot_sync(0xffffffffu, gt);
+      const uint32_t me = __ballot_sync(0xffffffffu, eq);
+      const uint32_t below = (1u << lane) - 1u;
+      if (gt) cand[gpos + __popc(mg & below)] = compose(key, imap ? imap[e] : e);
+      if (eq) {
+        const uint32_t r = epos + __popc(me & below);
+        if (r < kneed) cand[G + r] = compose(key, imap ? imap[e] : e);
+      }
+      gpos += __popc(mg);
+      epos += __popc(me);
     }
     C = target;
     cut = thr >> (32 - kScoreHistBits);
     btop = 0;
-    for (int e = t; e < n; e += kSelThreads) btop = max(btop, keys[e] >> (32 - kScoreHistBits));
+    for (int e = t; e < n; e += NT) btop = max(btop, keys[e] >> (32 - kScoreHistBits));
     uint32_t lo_dummy = 0xffffffffu;
     if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; }
     __syncthreads();
-    block_minmax(lo_dummy, btop, red);
+    block_minmax<NT>(lo_dummy, btop, red);
   }
   __syncthreads();
   // keys are dead from here on: their space holds the sorted pairs
-  if (!group_sort_desc<kSelThreads>(cand, C, sorted, hist, cut, btop, warp_sums, s_flag)) {
-    int sortn = kSelThreads;
+  if (C > 0 && !group_sort_adaptive<NT>(cand, C, sorted, hist,
+                               reinterpret_cast<uint8_t*>(rbuf) + RC::kAuxOff, cut, btop,
+                               warp_sums, s_flag, s_nsub)) {
+    int sortn = NT;
     while ((uint32_t)sortn < C) sortn <<= 1;
-    for (int i = t; i < sortn; i += kSelThreads) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
+    for (int i = t; i < sortn; i += NT) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
     __syncthreads();
-    switch (sortn / kSelThreads) {   // C <= kRowCandCap <= 16 * kSelThreads
-      case 1: sort_buf_desc_e<1, kSelThreads>(sorted); break;
-      case 2: sort_buf_desc_e<2, kSelThreads>(sorted); break;
-      case 4: sort_buf_desc_e<4, kSelThreads>(sorted); break;
-      case 8: sort_buf_desc_e<8, kSelThreads>(sorted); break;
-      default: sort_buf_desc_e<16, kSelThreads>(sorted); break;
-    }
+    row_bitonic<NT, RC::kEMax>(sorted, sortn);
   }
-  for (int i = t; i < topk; i += kSelThreads) {
+  for (int i = t; i < topk; i += NT) {
     const int64_t o = row * topk + i;
     if ((uint32_t)i < target) {
       const uint64_t v = sorted[i];
@@ -799,6 +852,24 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_row_kernel(
       if (vals) vals[o] = __int_as_float(0xff800000);
     }
   }
+}
+
+template <int NT, int CAP, int MINB>
+cudaError_t launch_row(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
+                       const int32_t* gather_len, const int32_t* index_map, int rows, int topk,
+                       int32_t* idx, float* vals, cudaStream_t st) {
+  using RC = RowCfg<NT, CAP>;
+  cudaError_t e = cudaFuncSetAttribute(topk_row_kernel<NT, CAP, MINB>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::kSmem);
+  if (e != cudaSuccess) return e;
+  for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
+    const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
+    topk_row_kernel<NT, CAP, MINB><<<(unsigned)nr, NT, RC::kSmem, st>>>(
+        scores, stride, pos, L, gather_len, index_map, topk, idx, vals, row0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -857,19 +928,18 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
   (void)status;
   const int sortn = topk_sort_size(topk);
   const int64_t maxlen = gather_len ? stride : L;
-  if (maxlen <= kRowCap && topk <= kRowCandCap) {
-    const size_t smem = (size_t)(kRowCap / 2 + kRowCandCap) * sizeof(uint64_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_row_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
-      const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
-      topk_row_kernel<<<(unsigned)nr, kSelThreads, smem, st>>>(scores, stride, pos, L, gather_len,
-                                                               index_map, topk, idx, vals, row0);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+  if (maxlen <= kRowCap && topk <= 8192) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (topk <= 3072 && rows >= 2 * sms)
+      return launch_row<256, 3072, 2>(scores, stride, pos, L, gather_len, index_map, rows, topk,
+                                      idx, vals, st);
+    if (rows >= sms)
+      return launch_row<512, 8192, 1>(scores, stride, pos, L, gather_len, index_map, rows, topk,
+                                      idx, vals, st);
+    return launch_row<1024, 8192, 1>(scores, stride, pos, L, gather_len, index_map, rows, topk,
+                                     idx, vals, st);
   }
   const int G = cluster_size_for(maxlen, sortn);
   if (G > 0) {

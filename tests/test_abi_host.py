@@ -67,6 +67,10 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert c.misa_pool_keys(null, 1, 1024, 64, 64, null, null) == 2
     # B < 1
     assert c.misa_pool_keys(null, 1, 1024, 128, 0, null, null) == 1
+    # refresh range outside [0, L] or reversed
+    assert c.misa_pool_keys_range(null, 1, 1024, 128, 64, 10, 5, null, null) == 1
+    assert c.misa_pool_keys_range(null, 1, 1024, 128, 64, -1, 5, null, null) == 1
+    assert c.misa_pool_keys_range(null, 1, 1024, 128, 64, 0, 1025, null, null) == 1
     # h > H
     assert c.misa_route_heads(null, null, null, null, null, 1, 1, 8, 128, 1024, 64, 9, null,
                               null, null, 0, null) == 1

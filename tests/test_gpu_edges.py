@@ -48,6 +48,8 @@ CASES = {
     "B_larger_than_L": dict(B=1024, L=300),
     "many_rows": dict(nseq=3, T=150, L=700, topk=50, kprime=100),
     "max_topk": dict(nseq=1, T=2, L=20000, topk=16384, kprime=16384, B=128),
+    # re-rank over more candidates than the row top-k keeps resident (16384 > 8192)
+    "dagger_wide_kprime": dict(nseq=1, T=2, L=20000, topk=2048, kprime=16384, B=128),
     # many queries per sequence: tensor-core router and query-block scorer
     "blocks_two_seqs_H16": dict(nseq=2, T=64, L=1000, H=16, h=4, topk=64, kprime=128),
     "blocks_H64_B32": dict(nseq=1, T=40, L=3000, H=64, h=8, B=32, topk=128, kprime=256),
@@ -176,3 +178,116 @@ def test_tied_long_rows_exact_fallback(M):
         didx = M.dsa_score_topk(q, w, k, pos, kk, return_vals=False)
         ref = torch.arange(kk, dtype=torch.int32).expand(2, 1, kk)
         assert torch.equal(idx.cpu(), ref) and torch.equal(didx.cpu(), ref), kk
+
+
+def test_dagger_candidates_any_order_with_repeats(M):
+    """Eq. (12) re-scores the set Omega_t: candidates given shuffled, with repeated ids
+    and empty slots, re-rank exactly like the oracle on the distinct ids."""
+    import oracle.misa_oracle as orc
+    from tests import tolerance as tl
+    wl = _wl(nseq=2, T=3, L=2000, topk=64, kprime=400)
+    x = make_inputs(wl, seed=21)
+    rng = np.random.default_rng(8)
+    cand = np.full((wl.nseq, wl.T, wl.kprime), -1, dtype=np.int32)
+    for n in range(wl.nseq):
+        for t in range(wl.T):
+            P = int(x.pos[n, t]) + 1
+            ids = rng.choice(P, size=300, replace=False)
+            rep = rng.choice(ids, size=60)                 # repeated ids
+            row = np.concatenate([ids, rep, np.full(40, -1)]).astype(np.int32)
+            cand[n, t] = rng.permutation(row)
+    q, w, k, pos = gpu_path.to_device(x)
+    idx, vals = M.misa_dagger_rerank(q, w, k, pos, torch.from_numpy(cand).to(q.device), wl.topk)
+    M.misa_check_device_status(q.device)
+    idx, vals = idx.cpu().numpy(), vals.cpu().numpy()
+    for n in range(wl.nseq):
+        kk = orc.bf16_bits_to_f64(x.k_bits[n])
+        for t in range(wl.T):
+            P = int(x.pos[n, t]) + 1
+            q_t = orc.bf16_bits_to_f64(x.q_bits[n, t])
+            d_ref = orc.dense_scores(q_t, x.w[n, t].astype(np.float64), kk, P)
+            c = np.unique(cand[n, t][cand[n, t] >= 0])
+            assert len(set(idx[n, t].tolist())) == wl.topk
+            tl.check_selection(idx[n, t], d_ref[c], wl.topk, what=f"dagger {n},{t}", ids=c)
+            tl.check_order(idx[n, t], vals[n, t], what=f"dagger order {n},{t}")
+            tl.check_scores(vals[n, t], d_ref[idx[n, t]], what=f"dagger vals {n},{t}")
+
+
+def test_pool_keys_range_refreshes_only_changed_blocks(M):
+    """Eq. (4) kept up to date: after keys in a token range change, the refresh rewrites
+    exactly the blocks meeting that range; the result equals a full re-pool bit for bit
+    (same kernel arithmetic) and the oracle's pooled keys within tolerance."""
+    import oracle.misa_oracle as orc
+    from tests import tolerance as tl
+    B = 64
+    wl = _wl(nseq=3, T=1, L=1000, B=B)
+    x = make_inputs(wl, seed=17)
+    _, _, k, _ = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, B)
+    rng = np.random.default_rng(4)
+    for s0, s1 in ((130, 131), (990, 1000), (0, 64), (300, 700), (999, 1000), (500, 500)):
+        new = rng.standard_normal((wl.nseq, s1 - s0, 128)).astype(np.float32) / np.sqrt(128)
+        x.k_bits[:, s0:s1] = fp32_to_bf16_bits(new)
+        _, _, k, _ = gpu_path.to_device(x)
+        b0, b1 = s0 // B, -(-s1 // B)
+        kp[:, :b0] = 7.0   # blocks outside the range must not be written
+        kp[:, b1:] = 7.0
+        M.misa_pool_keys_range(k, B, kp, s0, s1)
+        full = M.misa_pool_keys(k, B)
+        got = kp.cpu().numpy()
+        assert np.all(got[:, :b0] == 7.0) and np.all(got[:, b1:] == 7.0), (s0, s1)
+        assert torch.equal(kp[:, b0:b1], full[:, b0:b1]), (s0, s1)
+        for n in range(wl.nseq):
+            ref = orc.pool_keys(orc.bf16_bits_to_f64(x.k_bits[n]), B)
+            for b in range(b0, b1):
+                tl.check_scores(got[n, b], ref[b], what=f"block {n},{b} after [{s0},{s1})")
+        kp = full
+
+
+def test_decode_with_kept_pooled_keys(M):
+    """A decode loop that appends one key per step and refreshes only its block routes
+    and selects exactly like re-pooling every step."""
+    B = 64
+    wl = _wl(nseq=2, T=1, L=700, B=B, topk=64, kprime=128)
+    x = make_inputs(wl, seed=23)
+    q, w, k, pos = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, B)
+    for p in range(600, 700, 7):
+        pos.fill_(p)
+        x.k_bits[:, p] = fp32_to_bf16_bits(
+            np.random.default_rng(p).standard_normal((wl.nseq, 128)).astype(np.float32) / 12)
+        _, _, k, _ = gpu_path.to_device(x)
+        M.misa_pool_keys_range(k, B, kp, p, p + 1)
+        full = M.misa_pool_keys(k, B)
+        assert torch.equal(kp, full), p
+        h1 = M.misa_route_heads(q, w, k, kp, pos, B, wl.h)
+        h2 = M.misa_route_heads(q, w, k, full, pos, B, wl.h)
+        assert torch.equal(h1, h2), p
+
+
+@pytest.mark.parametrize("T,L,topk", [(300, 5000, 3000), (300, 10000, 8192)])
+def test_tied_rows_many_queries(M, T, L, topk):
+    """Many rows of equal scores longer than the row top-k's candidate room: the crowded
+    cutoff takes the exact radix select and returns the lowest indices."""
+    wl = _wl(nseq=1, T=T, L=L, H=8, h=3, topk=topk, kprime=topk)
+    x = make_inputs(wl, seed=6)
+    x.k_bits[:] = fp32_to_bf16_bits(np.full((128,), 0.05, dtype=np.float32))[None, None, :]
+    q, w, k, pos = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, wl.B)
+    heads = M.misa_route_heads(q, w, k, kp, pos, wl.B, wl.h)
+    idx = M.misa_score_topk(q, w, k, heads, pos, topk, return_vals=False)
+    ref = torch.arange(topk, dtype=torch.int32).expand(1, T, topk)
+    assert torch.equal(idx.cpu(), ref)
+
+
+def test_tied_candidates_exact_rerank(M):
+    """12000 tied candidates re-ranked to 8192: exact fallback over an index map."""
+    wl = _wl(nseq=2, T=1, L=13000, H=8, h=3, topk=8192, kprime=12000)
+    x = make_inputs(wl, seed=7)
+    x.k_bits[:] = fp32_to_bf16_bits(np.full((128,), 0.05, dtype=np.float32))[None, None, :]
+    q, w, k, pos = gpu_path.to_device(x)
+    rng = np.random.default_rng(3)
+    cand = np.stack([rng.permutation(12000) for _ in range(2)]).astype(np.int32)[:, None, :]
+    idx, _ = M.misa_dagger_rerank(q, w, k, pos, torch.from_numpy(cand).to(q.device), 8192)
+    ref = torch.arange(8192, dtype=torch.int32).expand(2, 1, 8192)
+    assert torch.equal(idx.cpu(), ref)

@@ -140,15 +140,17 @@ def algorithmic_flops_score(wl) -> float:
 
 
 def algorithmic_bytes_score(wl) -> float:
-    """Bytes the routed score + top-k call must move: every key of every query's prefix
-    (256 B per token per query row -- decode rows do not share keys), the routed query
-    vectors, and the selected indices/values."""
+    """Bytes the routed scoring kernel (misa_score_rows, the scorer misa_score_topk runs)
+    must move: every key of every query's prefix, 256 B per token (decode rows do not
+    share keys; the queries of a prefill sequence share its keys), each query's routed
+    head vectors, weights and head ids (h * (256 + 4 + 4) B), and one fp32 score written
+    per query x prefix-token."""
     P = wl.positions().astype(np.int64) + 1
     if wl.T == 1:
         keys = float(P.sum()) * wl.d * 2
     else:
-        keys = float(wl.nseq) * wl.L * wl.d * 2   # one sequence's keys shared by its queries
-    return keys + wl.rows * (wl.h * wl.d * 2 + wl.h * 4 + wl.H * 4) + wl.rows * wl.topk * 8
+        keys = float(wl.nseq) * wl.L * wl.d * 2
+    return keys + wl.rows * wl.h * (wl.d * 2 + 4 + 4) + 4.0 * wl.query_prefix_tokens()
 
 
 def run_reference(args, wl):

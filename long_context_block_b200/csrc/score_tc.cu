@@ -25,6 +25,13 @@
 // MISA_ERR_DEVICE_TIMEOUT, lets its in-flight copies and MMAs finish, frees TMEM and
 // returns.  In decode form the epilogue can also build a per-row histogram of the score
 // keys for the top-k that follows.
+//
+// Gather mode (MISA-dagger fine stage, Eq. 12): a row scores its own list of candidate
+// tokens instead of its prefix.  Its key rows are scattered, so the producer warp copies
+// them with cp.async, 16 bytes per lane and two rows per warp step, straight into the
+// swizzled tile layout; each lane's arrival on the stage barrier fires when its copies
+// have landed, and the MMA thread fences the async proxy before reading the tile.  (A
+// TMA row gather, four rows per instruction, measured at about half this rate.)
 #include <cuda.h>
 
 #include <mutex>

@@ -78,20 +78,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Row gather: four rows y0..y3 of a 2-D map whose box is (x extent, 1 row) land one
-// after another at dst, as rows of a tiled load would (the swizzle follows the
-// destination address, so dst must sit at the rows' place in a 1024-byte-aligned tile).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y0, int32_t y1, int32_t y2,
-                                            int32_t y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
-      "r"(y2), "r"(y3)
-      : "memory");
-}
-
 // 16-byte asynchronous copy global -> shared memory (L2 only), and the arrival on `bar`
 // that fires once every cp.async this thread issued before it has landed (the barrier's
 // expected count includes that arrival: .noinc).  The data is written through the

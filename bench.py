@@ -295,6 +295,20 @@ def run_cuda(args, wl):
         M.misa_route_heads(q, w, k, kp[i % 2], pos, wl.B, wl.h, heads=heads)
         M.misa_score_topk(q, w, k, heads, pos, wl.topk, idx=idx, vals=vals)
 
+    if args.only:
+        # one path's steps and nothing else (for profiler captures); prints no bench line
+        fn = {"misa": misa_step, "dagger": dagger_step, "dsa": dsa_step}[args.only]
+        for i in range(args.warmup + args.steps):
+            fn(i)
+        torch.cuda.synchronize()
+        M.misa_check_device_status(dev)
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"only": args.only, "workload": wl.name,
+                              "steps": args.warmup + args.steps}))
+        return 0
+
     def barrier():
         if world > 1:
             dist.barrier()
@@ -441,8 +455,12 @@ def main():
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override an integer field of the workload (e.g. T=8192), for "
                          "smaller profiling runs; the JSON line names the result")
+    ap.add_argument("--only", choices=["misa", "dagger", "dsa"],
+                    help="run only this path's warm-up + timed steps, untimed, and print no "
+                         "bench line (for profiler captures)")
     args = ap.parse_args()
-    args.warmup = max(3, args.warmup)
+    if not args.only:
+        args.warmup = max(3, args.warmup)
     wl = WORKLOADS[args.workload]
     for kv in args.set:
         field, value = kv.split("=", 1)

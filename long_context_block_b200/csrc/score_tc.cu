@@ -139,7 +139,7 @@ struct Units {
   __device__ __forceinline__ int t0(int u) const { return (u % ublk) * QB; }
 };
 
-template <int HS, int QB>
+template <int HS, int QB, bool kGather>
 __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ wsel, const int32_t* __restrict__ pos,
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
   if (tid == 0) {
     // a gathered tile completes with one cp.async arrival per producer lane
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], gidx ? 32 : 1);
+      mbar_init(&full[s], kGather ? 32 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < C::kQBufs; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
@@ -204,61 +204,101 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    // The whole warp walks the loop (waits are polled by lane 0 and broadcast); lane 0
-    // issues the tile loads, or in gather mode every lane gathers four key rows.
     int issued = 0, qissued = 0, wissued = 0;
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_q);
-    }
-    int u = u_first;
-    Seg sg;
-    bool ok = true;
-    while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
-      const int slot = qissued % C::kQBufs;
-      if (!warp_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status)) break;
-      uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
+    if constexpr (!kGather) {
+      // lane 0 streams each unit's q tile, weights and prefix key tiles by TMA
       if (lane == 0) {
-        mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
-        tma_load_2d(qb, &tm_q, &qfull[slot], 0, sg.u * N);
-        tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
-      }
-      const int wslot = qissued % C::kWBufs;
-      if (!warp_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status)) {
-        ++qissued;
-        break;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&wfull[wslot], C::kWBytes);
-        bulk_load(base + C::kWBase + wslot * C::kWBytes, wsel + (int64_t)sg.u * N, C::kWBytes,
-                  &wfull[wslot]);
-      }
-      ++qissued;
-      ++wissued;
-      const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
-      // gather mode (QB == 1, unit = row): the row's token list and its length; lane l
-      // gathers keys 4l .. 4l+3 of a tile, whose ids it loads kIdAhead tiles early
-      const int32_t* ids = gidx ? gidx + (int64_t)sg.u * out_stride : nullptr;
-      const int cnt = gidx ? min(max(glen[sg.u], 0), (int)out_stride) : 0;
-      int32_t rq[kIdAhead][4];
-      auto fetch_ids = [&](int jj, int32_t(&r)[4]) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = jj * kTileKeys + 4 * lane + i;
-          int32_t id = c < cnt ? ids[c] : 0;   // padding keys are masked by the epilogue
-          if (id < 0 || id >= L) id = 0;
-          r[i] = (int32_t)(y0 + id);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_q);
+        int u = u_first;
+        Seg sg;
+        bool ok = true;
+        while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
+          const int slot = qissued % C::kQBufs;
+          if (!mbar_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status,
+                         kWaitCycles))
+            break;
+          uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
+          mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
+          tma_load_2d(qb, &tm_q, &qfull[slot], 0, sg.u * N);
+          tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
+          const int wslot = qissued % C::kWBufs;
+          if (!mbar_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status,
+                         kWaitCycles)) {
+            ++qissued;
+            break;
+          }
+          mbar_arrive_expect_tx(&wfull[wslot], C::kWBytes);
+          bulk_load(base + C::kWBase + wslot * C::kWBytes, wsel + (int64_t)sg.u * N, C::kWBytes,
+                    &wfull[wslot]);
+          ++qissued;
+          ++wissued;
+          const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
+          for (int j = sg.a; j < sg.b; ++j) {
+            const int s = issued % C::kStages;
+            if (!mbar_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status,
+                           kWaitCycles)) {
+              ok = false;
+              break;
+            }
+            uint8_t* kb = base + C::kStageBase + s * kKeyTileBytes;
+            mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
+            const int32_t y = (int32_t)(y0 + (int64_t)j * kTileKeys);
+            tma_load_2d(kb, &tm_k, &full[s], 0, y);
+            tma_load_2d(kb + kKeyHalfBytes, &tm_k, &full[s], 64, y);
+            ++issued;
+          }
         }
-      };
-      if (ids) {
+      }
+    } else {
+      // gather mode: the whole warp walks the loop (waits are polled by lane 0 and
+      // broadcast); lane 0 loads q and the weights, every lane copies key rows
+      if (lane == 0) tma_prefetch_desc(&tm_q);
+      int u = u_first;
+      Seg sg;
+      bool ok = true;
+      while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
+        const int slot = qissued % C::kQBufs;
+        if (!warp_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status)) break;
+        uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
+          tma_load_2d(qb, &tm_q, &qfull[slot], 0, sg.u * N);
+          tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
+        }
+        const int wslot = qissued % C::kWBufs;
+        if (!warp_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status)) {
+          ++qissued;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&wfull[wslot], C::kWBytes);
+          bulk_load(base + C::kWBase + wslot * C::kWBytes, wsel + (int64_t)sg.u * N, C::kWBytes,
+                    &wfull[wslot]);
+        }
+        ++qissued;
+        ++wissued;
+        const int64_t y0 = (int64_t)geo.seq(sg.u) * L;
+        // unit = row: its token list and length; lane l gathers keys 4l .. 4l+3 of a tile,
+        // whose ids it loads kIdAhead tiles early
+        const int32_t* ids = gidx + (int64_t)sg.u * out_stride;
+        const int cnt = min(max(glen[sg.u], 0), (int)out_stride);
+        int32_t rq[kIdAhead][4];
+        auto fetch_ids = [&](int jj, int32_t(&r)[4]) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = jj * kTileKeys + 4 * lane + i;
+            int32_t id = c < cnt ? ids[c] : 0;   // padding keys are masked by the epilogue
+            if (id < 0 || id >= L) id = 0;
+            r[i] = (int32_t)(y0 + id);
+          }
+        };
 #pragma unroll
         for (int d = 0; d < kIdAhead; ++d)
           if (sg.a + d < sg.b) fetch_ids(sg.a + d, rq[d]);
-      }
-      for (int j = sg.a; j < sg.b; ++j) {
-        const int s = issued % C::kStages;
-        int32_t r[4];
-        if (ids) {
+        for (int j = sg.a; j < sg.b; ++j) {
+          const int s = issued % C::kStages;
+          int32_t r[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) r[i] = rq[0][i];
 #pragma unroll
@@ -266,18 +306,16 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 #pragma unroll
             for (int i = 0; i < 4; ++i) rq[d][i] = rq[d + 1][i];
           if (j + kIdAhead < sg.b) fetch_ids(j + kIdAhead, rq[kIdAhead - 1]);
-        }
-        if (!warp_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status)) {
-          ok = false;
-          break;
-        }
-        uint8_t* kb = base + C::kStageBase + s * kKeyTileBytes;
-        if (ids) {
+          if (!warp_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
           // 64 warp-wide steps, two key rows each: lanes 0-15 copy row 2i, lanes 16-31 row
           // 2i+1, 16 bytes per lane, into the 128-byte-swizzled halves of the tile.  Row
           // 4m+e's id sits in lane m's r[e].
           const int c = lane & 15, odd = lane >> 4;
-          const uint32_t kb_s = smem_u32(kb) + (uint32_t)((c >> 3) * kKeyHalfBytes);
+          const uint32_t kb_s = smem_u32(base + C::kStageBase + s * kKeyTileBytes) +
+                                (uint32_t)((c >> 3) * kKeyHalfBytes);
 #pragma unroll
           for (int i = 0; i < kTileKeys / 2; ++i) {
             const int32_t ya = __shfl_sync(0xffffffffu, r[2 * (i & 1)], i >> 1);
@@ -287,13 +325,8 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
             cp_async16(dst, kraw + (int64_t)(odd ? yb : ya) * kHeadDim + c * 8);
           }
           cp_async_mbar_arrive(&full[s]);
-        } else if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
-          const int32_t y = (int32_t)(y0 + (int64_t)j * kTileKeys);
-          tma_load_2d(kb, &tm_k, &full[s], 0, y);
-          tma_load_2d(kb + kKeyHalfBytes, &tm_k, &full[s], 64, y);
+          ++issued;
         }
-        ++issued;
       }
     }
     __syncthreads();   // (A) every role has left its loop
@@ -329,7 +362,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
             break;
           }
           tc_fence_after();
-          if (gidx) fence_proxy_async_smem();   // gathered tile was written by cp.async
+          if constexpr (kGather) fence_proxy_async_smem();   // tile written by cp.async
           const uint32_t kaddr = smem0 + C::kStageBase + s * kKeyTileBytes;
           const uint32_t d = tmem_base + (uint32_t)(acc * C::kAccStride);
 #pragma unroll
@@ -378,9 +411,10 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 #pragma unroll
       for (int q = 0; q < kQPerWarp; ++q) {
         const int t = tq0 + q0 + q;
-        P[q] = t >= geo.T ? 0
-               : gidx  ? min(max(glen[sg.u], 0), (int)out_stride)
-                       : prefix_len(pos, (int64_t)n * geo.T + t, L, nullptr);
+        if constexpr (kGather)
+          P[q] = t >= geo.T ? 0 : min(max(glen[sg.u], 0), (int)out_stride);
+        else
+          P[q] = t < geo.T ? prefix_len(pos, (int64_t)n * geo.T + t, L, nullptr) : 0;
       }
       // this warp's queries are consecutive rows of the output
       float* obase = out + ((int64_t)n * geo.T + min(tq0 + q0, geo.T - 1)) * out_stride;
@@ -556,20 +590,20 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t nrows, uint32_t box_rows
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int HS, int QB>
+template <int HS, int QB, bool kGather>
 cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float* wg,
                        const int32_t* pos, const int32_t* tile_off, int units, Units geo,
                        int64_t L, float* out, int64_t out_stride, int* status, uint32_t* hist,
                        const int32_t* gidx, const int32_t* glen, const uint16_t* kraw,
                        cudaStream_t st) {
   using C = Cfg<HS, QB>;
-  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB>,
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB, kGather>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  score_tc_kernel<HS, QB><<<sms, C::kThreads, C::kSmemBytes, st>>>(
+  score_tc_kernel<HS, QB, kGather><<<sms, C::kThreads, C::kSmemBytes, st>>>(
       tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist, gidx, glen, kraw);
   return cudaGetLastError();
 }
@@ -646,8 +680,23 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
     return cudaErrorInvalidValue;
 #define MISA_TC_CASE(HS_, QB_)                                                                  \
   if (p.HS == HS_ && p.QB == QB_)                                                               \
-    return launch_cfg<HS_, QB_>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, \
-                                hist, gidx, glen, k, st);
+    return launch_cfg<HS_, QB_, false>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, \
+                                       status, hist, nullptr, nullptr, k, st);
+#define MISA_TC_GATHER_CASE(HS_)                                                                \
+  if (p.HS == HS_)                                                                              \
+    return launch_cfg<HS_, 1, true>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride,    \
+                                    status, nullptr, gidx, glen, k, st);
+  if (gather) {
+    MISA_TC_GATHER_CASE(16)
+    MISA_TC_GATHER_CASE(32)
+    MISA_TC_GATHER_CASE(48)
+    MISA_TC_GATHER_CASE(64)
+    MISA_TC_GATHER_CASE(80)
+    MISA_TC_GATHER_CASE(96)
+    MISA_TC_GATHER_CASE(112)
+    MISA_TC_GATHER_CASE(128)
+    return cudaErrorInvalidValue;
+  }
   MISA_TC_CASE(16, 1)
   MISA_TC_CASE(32, 1)
   MISA_TC_CASE(48, 1)
@@ -662,6 +711,7 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
   MISA_TC_CASE(64, 4)
   MISA_TC_CASE(128, 2)
 #undef MISA_TC_CASE
+#undef MISA_TC_GATHER_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -225,7 +225,7 @@ static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* 
       MISA_TRY(cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, sc, L,
                                            tc_scratch, status, hist, st)));
       return cuda_status(launch_topk_hist(sc, L, pos, L, hist, cand, gcount, (int)rows, topk, idx,
-                                          vals, st));
+                                          vals, status, st));
     }
     MISA_TRY(cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, sc, L, tc_scratch,
                                          status, nullptr, st)));

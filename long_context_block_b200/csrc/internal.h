@@ -83,14 +83,16 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
                         const int32_t* gather_len, const int32_t* index_map, int rows,
                         int topk, int32_t* idx, float* vals, int* status, cudaStream_t st);
 
-// K5 for long rows with a histogram of their scores (topk.cu): the bins at or above the
-// bin of the row's k-th largest score are split into groups of output positions; a
-// scatter pass appends every candidate to its group's buffer and one CTA per group sorts
-// and writes it.  hist: rows x kScoreHistBins (filled by the scorer); gcount: rows x 16
-// (zeroed by the caller, directly after hist); cand: topk_hist_ws_bytes layout.
+// K5 for long rows with a histogram of their scores (topk.cu).  Rows that fit one SM's
+// shared memory (up to 40960 scores, k <= 3072) are selected by one CTA per row that takes
+// the cutoff bin from the histogram; longer rows split the bins at or above the cutoff
+// into groups of output positions: a scatter pass appends every candidate to its group's
+// buffer and one CTA per group sorts and writes it.  hist: rows x kScoreHistBins (filled
+// by the scorer); gcount: rows x 16 (zeroed by the caller, directly after hist); cand:
+// topk_hist_ws_bytes layout.
 cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
                              const uint32_t* hist, uint64_t* cand, uint32_t* gcount, int rows,
-                             int topk, int32_t* idx, float* vals, cudaStream_t st);
+                             int topk, int32_t* idx, float* vals, int* status, cudaStream_t st);
 // Scratch of the histogram path: histogram, group counts, group buffers (256-aligned each).
 size_t topk_hist_ws_bytes(int64_t rows);
 

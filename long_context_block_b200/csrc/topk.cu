@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "groupsort.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -606,20 +607,25 @@ __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
 }
 
 // ---------------------------------------------------------------- row-resident form
-// Rows of up to kRowCap scores and k <= CAP: one CTA of NT threads per row keeps the row's
-// keys in shared memory, finds the cutoff bin with a shared-memory histogram of the top
-// kScoreHistBits key bits, compacts the candidates (bins at or above it) and sorts them
-// with the counting sort.  A crowded cutoff (more than CAP candidates) takes an exact
-// radix select over the resident keys instead.  Three shapes: 256 threads and 3072
-// candidates (two CTAs per SM, many rows, k <= 3072), 512 or 1024 threads and 8192
-// candidates (one CTA per SM; 1024 threads when there are too few rows to fill the SMs).
+// Rows of up to ROWCAP scores and k <= CAP: one CTA of NT threads per row copies the row
+// into shared memory with one bulk asynchronous copy (plain loads for the at most three
+// scores on either side of its 16-byte-aligned interior), turns the scores into keys in
+// place, finds the cutoff bin with a histogram of the top kScoreHistBits key bits (or
+// takes the one the scorer built), compacts the candidates (bins at or above it) and
+// sorts them with the counting sort.  A crowded cutoff (more than CAP candidates) takes
+// an exact radix select over the resident keys instead.  Shapes: 256 threads, 3072
+// candidates, 16K rows (two CTAs per SM: many rows, k <= 3072); 512 or 1024 threads, 8192
+// candidates, 16K rows (one CTA per SM; 1024 threads when rows are too few to fill the
+// SMs); 1024 threads, 3072 candidates, 40K rows (long decode rows).
 constexpr int kRowCap = 16384;
-constexpr int kRowLoadUnroll = 8;
+constexpr int kLongRowCap = 40960;
+constexpr long long kRowWaitCycles = 4000000000LL;
 
-template <int NT, int CAP>
+template <int NT, int CAP, int ROWCAP>
 struct RowCfg {
-  // keys [kRowCap] u32, later the sorted pairs [<= CAP] u64, then the candidates [CAP] u64
-  static constexpr int kKeyPairs = kRowCap / 2 > CAP ? kRowCap / 2 : CAP;
+  // keys [ROWCAP] u32 (+16 bytes to align the bulk copy), later the sorted pairs [<= CAP]
+  // u64, then the candidates [CAP] u64
+  static constexpr int kKeyPairs = (ROWCAP * 4 + 16) / 8 > CAP ? (ROWCAP * 4 + 16) / 8 : CAP;
   // the adaptive sort's bin tables sit in the key space the sorted pairs leave free, or
   // after the candidates
   static constexpr bool kAuxInKeys = (kKeyPairs - CAP) * 8 >= kAdaptiveAuxBytes;
@@ -629,7 +635,7 @@ struct RowCfg {
   static constexpr int kEMax = CAP <= NT ? 1 : CAP <= 2 * NT ? 2 : CAP <= 4 * NT ? 4
                                : CAP <= 8 * NT ? 8 : 16;
   static constexpr int kBinsPer = 2048 / NT;   // radix-select bins per thread
-  static_assert(CAP <= 16 * NT && 2048 % NT == 0, "row kernel shape");
+  static_assert(CAP <= 16 * NT && 2048 % NT == 0 && ROWCAP < 65536, "row kernel shape");
 };
 
 template <int NT>
@@ -665,20 +671,21 @@ __device__ __forceinline__ void row_bitonic(uint64_t* sorted, int sortn) {
   }
 }
 
-template <int NT, int CAP, int MINB>
+template <int NT, int CAP, int ROWCAP, int MINB>
 __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
-    const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map, int topk,
-    int32_t* __restrict__ idx, float* __restrict__ vals, int64_t row0) {
-  using RC = RowCfg<NT, CAP>;
-  extern __shared__ uint64_t rbuf[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(rbuf);          // [kRowCap] keys, then
-  uint64_t* sorted = rbuf;                                     //   [CAP] sorted pairs
+    const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map,
+    const uint32_t* __restrict__ ghist, int topk, int32_t* __restrict__ idx,
+    float* __restrict__ vals, int* status, int64_t row0) {
+  using RC = RowCfg<NT, CAP, ROWCAP>;
+  extern __shared__ __align__(128) uint64_t rbuf[];
+  uint64_t* sorted = rbuf;                                     // [CAP] sorted pairs (later)
   uint64_t* cand = rbuf + RC::kKeyPairs;                       // [CAP] candidates
   __shared__ __align__(16) uint32_t hist[kSubBucketWords];     // histogram, then buckets
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t red[2];
   __shared__ uint32_t s_cut, s_total, s_big, s_fill, s_flag, s_digit, s_above, s_top, s_nsub;
+  __shared__ __align__(8) uint64_t lbar;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t row = row0 + blockIdx.x;
   const int n = gather_len ? gather_len[row] : prefix_len(pos, row, L, nullptr);
@@ -686,21 +693,44 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   const float* x = scores + row * stride;
   const int32_t* imap = index_map ? index_map + row * stride : nullptr;
 
-  for (int b = t; b < kScoreHistBins; b += NT) hist[b] = 0;
+  // keys[e] holds score e: the 16-byte-aligned interior of the row arrives by one bulk
+  // copy, to a shared address that is 16-byte aligned too (keys starts `hb` bytes in)
+  const uint32_t hb = (uint32_t)(reinterpret_cast<uintptr_t>(x) & 15u);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(rbuf) + hb);
+  const int h0 = min((int)(((16u - hb) & 15u) >> 2), n);   // scores before the interior
+  const int nbulk = ((n - h0) >> 2) << 2;                   // interior scores
+  if (t == 0) {
+    sm100::mbar_init(&lbar, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (t == 0 && nbulk > 0) {
+    sm100::mbar_arrive_expect_tx(&lbar, (uint32_t)nbulk * 4u);
+    sm100::bulk_load(keys + h0, x + h0, (uint32_t)nbulk * 4u, &lbar);
+  }
+  if (t < h0) keys[t] = __float_as_uint(x[t]);
+  if (t < 4 && h0 + nbulk + t < n) keys[h0 + nbulk + t] = __float_as_uint(x[h0 + nbulk + t]);
+  for (int b = t; b < kScoreHistBins; b += NT) hist[b] = (ghist && n > (int)target)
+                                                    ? ghist[row * kScoreHistBins + b] : 0u;
   if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; s_fill = 0; s_top = 0; }
-  for (int base = 0; base < n; base += NT * kRowLoadUnroll) {
-    float v[kRowLoadUnroll];
-#pragma unroll
-    for (int j = 0; j < kRowLoadUnroll; ++j) {
-      const int e = base + j * NT + t;
-      v[j] = e < n ? x[e] : 0.f;
+  if (nbulk > 0) {   // bounded wait for the copy; on expiry the row's result is void
+    long long t0 = clock64();
+    bool landed = true;
+    while (!sm100::mbar_try_wait(&lbar, 0)) {
+      if (clock64() - t0 > kRowWaitCycles) {
+        landed = false;
+        break;
+      }
     }
-#pragma unroll
-    for (int j = 0; j < kRowLoadUnroll; ++j) {
-      const int e = base + j * NT + t;
-      if (e < n) keys[e] = score_key(v[j]);
+    if (!landed) {   // record it, then give the copy one more bounded wait before going on
+      if (t == 0) set_status(status, MISA_ERR_DEVICE_TIMEOUT);
+      t0 = clock64();
+      while (!sm100::mbar_try_wait(&lbar, 0) && clock64() - t0 <= kRowWaitCycles) {
+      }
     }
   }
+  __syncthreads();
+  for (int e = t; e < n; e += NT) keys[e] = score_key(__uint_as_float(keys[e]));
   __syncthreads();
   uint32_t cut, btop, C;
   if ((uint32_t)n <= target) {
@@ -716,8 +746,10 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     btop = hi;
     C = (uint32_t)n;
   } else {
-    for (int e = t; e < n; e += NT) atomicAdd(&hist[keys[e] >> (32 - kScoreHistBits)], 1u);
-    __syncthreads();
+    if (!ghist) {
+      for (int e = t; e < n; e += NT) atomicAdd(&hist[keys[e] >> (32 - kScoreHistBits)], 1u);
+      __syncthreads();
+    }
     HistView<NT> hv;
     cut = hist_cutoff<NT>(hist, target, hv, warp_sums, s_cut, s_total, s_big);
     // highest occupied bin
@@ -854,18 +886,19 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   }
 }
 
-template <int NT, int CAP, int MINB>
+template <int NT, int CAP, int ROWCAP, int MINB>
 cudaError_t launch_row(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
-                       const int32_t* gather_len, const int32_t* index_map, int rows, int topk,
-                       int32_t* idx, float* vals, cudaStream_t st) {
-  using RC = RowCfg<NT, CAP>;
-  cudaError_t e = cudaFuncSetAttribute(topk_row_kernel<NT, CAP, MINB>,
+                       const int32_t* gather_len, const int32_t* index_map, const uint32_t* ghist,
+                       int rows, int topk, int32_t* idx, float* vals, int* status,
+                       cudaStream_t st) {
+  using RC = RowCfg<NT, CAP, ROWCAP>;
+  cudaError_t e = cudaFuncSetAttribute(topk_row_kernel<NT, CAP, ROWCAP, MINB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::kSmem);
   if (e != cudaSuccess) return e;
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
-    topk_row_kernel<NT, CAP, MINB><<<(unsigned)nr, NT, RC::kSmem, st>>>(
-        scores, stride, pos, L, gather_len, index_map, topk, idx, vals, row0);
+    topk_row_kernel<NT, CAP, ROWCAP, MINB><<<(unsigned)nr, NT, RC::kSmem, st>>>(
+        scores, stride, pos, L, gather_len, index_map, ghist, topk, idx, vals, status, row0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -882,7 +915,10 @@ int topk_sort_size(int topk) {
 
 cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
                              const uint32_t* hist, uint64_t* cand, uint32_t* gcount, int rows,
-                             int topk, int32_t* idx, float* vals, cudaStream_t st) {
+                             int topk, int32_t* idx, float* vals, int* status, cudaStream_t st) {
+  if (L <= kLongRowCap && topk <= 3072)
+    return launch_row<1024, 3072, kLongRowCap, 1>(scores, stride, pos, L, nullptr, nullptr, hist,
+                                                  rows, topk, idx, vals, status, st);
   dim3 sgrid((unsigned)((L + kScatterChunk - 1) / kScatterChunk), (unsigned)rows);
   topk_scatter_kernel<<<sgrid, kSelThreads, 0, st>>>(scores, stride, pos, L, hist, topk, cand,
                                                      gcount);
@@ -925,7 +961,6 @@ static int cluster_size_for(int64_t len, int sortn) {
 cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
                         const int32_t* gather_len, const int32_t* index_map, int rows,
                         int topk, int32_t* idx, float* vals, int* status, cudaStream_t st) {
-  (void)status;
   const int sortn = topk_sort_size(topk);
   const int64_t maxlen = gather_len ? stride : L;
   if (maxlen <= kRowCap && topk <= 8192) {
@@ -933,14 +968,17 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (topk <= 3072 && rows >= 2 * sms)
-      return launch_row<256, 3072, 2>(scores, stride, pos, L, gather_len, index_map, rows, topk,
-                                      idx, vals, st);
+      return launch_row<256, 3072, kRowCap, 2>(scores, stride, pos, L, gather_len, index_map,
+                                               nullptr, rows, topk, idx, vals, status, st);
     if (rows >= sms)
-      return launch_row<512, 8192, 1>(scores, stride, pos, L, gather_len, index_map, rows, topk,
-                                      idx, vals, st);
-    return launch_row<1024, 8192, 1>(scores, stride, pos, L, gather_len, index_map, rows, topk,
-                                     idx, vals, st);
+      return launch_row<512, 8192, kRowCap, 1>(scores, stride, pos, L, gather_len, index_map,
+                                               nullptr, rows, topk, idx, vals, status, st);
+    return launch_row<1024, 8192, kRowCap, 1>(scores, stride, pos, L, gather_len, index_map,
+                                              nullptr, rows, topk, idx, vals, status, st);
   }
+  if (maxlen <= kLongRowCap && topk <= 3072)
+    return launch_row<1024, 3072, kLongRowCap, 1>(scores, stride, pos, L, gather_len, index_map,
+                                                  nullptr, rows, topk, idx, vals, status, st);
   const int G = cluster_size_for(maxlen, sortn);
   if (G > 0) {
     const int64_t slice = (((maxlen + G - 1) / G) + 3) & ~int64_t(3);

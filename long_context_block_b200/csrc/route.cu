@@ -8,13 +8,16 @@
 // pooled-key tensor, and when the prefix ends inside a block that block's pooled
 // key is the mean of its valid keys only, computed here from the raw keys.
 //
-// One kernel, grid = (chunks of kRouteChunk blocks, query rows).  A CTA stages its
-// chunk of pooled keys in shared memory (fp32) and each thread keeps one head's query
-// vector in registers; G thread groups split the chunk's blocks.  It writes
+// One kernel, grid = (chunks of kRouteChunk blocks, query rows), for queries that do not
+// share a sequence with many others (decode).  A CTA stages the query's head vectors and
+// its chunk of pooled keys in shared memory and computes q_j . kp_b on the tensor cores
+// (mma.sync, bf16 operands, fp32 pooled keys split into hi + lo parts).  It writes
 // sum_b ReLU(q_j . kp_b) for its chunk to the workspace and bumps the row's counter;
 // the last CTA of a row to finish sums the chunk partials, applies |w_j| / M_t (common
 // to all blocks, so applied once), writes E and selects the top-h heads by repeated
 // warp arg-max.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -60,28 +63,49 @@ __device__ __forceinline__ void select_top_h(const float* ev, int H, int h, int3
   }
 }
 
-// Chunk of kRouteChunk blocks x up to 32*HG heads.  Thread (hp, bq) owns heads
-// hp + 32*m (m < HG) and blocks 4*bq .. 4*bq+3 of the chunk: a register-tiled
-// dot-product microkernel over d with q and pooled keys in shared memory (fp32).
-constexpr int kRouteThreads = 256;
-constexpr int kQStride = kHeadDim + 4;   // padded fp32 row: conflict-free 16-byte reads
+// One CTA = one (chunk of kCh blocks, query row): 4 warps; warp w takes the 16-head row
+// tiles w, w+4 (of ceil(H/16)).  The contraction S[j, b] = q_j . kp_b runs on the tensor
+// cores as mma.sync m16n8k16 with bf16 operands and fp32 accumulators: A = the query's
+// head vectors (bf16 as given), B = the chunk's pooled keys split into bf16 hi + lo
+// (hi = bf16(kp), lo = bf16(kp - hi)), so the two products reproduce the fp32 pooled key
+// to about 2^-16 relative.  Operands sit in shared memory as rows of 128 bf16 padded by
+// 16 bytes (fragment loads conflict-free).
+constexpr int kRouteThreads = 128;
+constexpr int kRowPad = kHeadDim + 8;   // bf16 elements per padded shared row
 
-template <int HG>
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int MT>   // 16-head row tiles per warp (ceil(ceil(H/16) / 4))
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
     const float* __restrict__ k_pool, const int32_t* __restrict__ pos, int T, int H,
     int64_t L, int B, int Mpool, float* __restrict__ partial, int nchunk, int* status,
     int64_t row0, const float* __restrict__ w, int h, int* __restrict__ counters,
     int32_t* __restrict__ heads, float* __restrict__ E) {
-  extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                                   // [32*HG][kQStride]
-  float* kp = sm + 32 * HG * kQStride;              // [kCh][kQStride]
-  __shared__ float red[kRouteThreads / 32][32 * HG];
+  extern __shared__ __align__(16) uint16_t rsm[];
+  uint16_t* qs = rsm;                                  // [16 * 4 * MT][kRowPad] bf16
+  uint16_t* khi = qs + 16 * 4 * MT * kRowPad;          // [kCh][kRowPad]
+  uint16_t* klo = khi + kCh * kRowPad;                 // [kCh][kRowPad]
+  __shared__ float kpart[kHeadDim];                    // partial block's pooled key
+  __shared__ float rsum[MISA_MAX_HEADS];
+  __shared__ float red[kRouteThreads / 32][32];
   __shared__ float ev[MISA_MAX_HEADS];
   __shared__ int s_last;
   const int64_t row = row0 + blockIdx.y;
   const int chunk = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = prefix_len(pos, row, L, chunk == 0 && tid == 0 ? status : nullptr);
   const int M = (P + B - 1) / B;
   const int Mfull = P / B;
@@ -89,80 +113,130 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   if (b0 >= M) return;
   const int nb = min(b0 + kCh, M) - b0;
   const int64_t n = row / T;
+  const int HT = 16 * 4 * MT;   // head rows staged (zero past H)
+  const bool has_part = Mfull < M && Mfull >= b0 && Mfull < b0 + nb;
 
-  // q rows of this query (bf16 -> fp32), zero rows past H
-  for (int e = tid; e < 32 * HG * (kHeadDim / 8); e += kRouteThreads) {
-    const int j = e / (kHeadDim / 8), c = e % (kHeadDim / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (j < H) v = reinterpret_cast<const uint4*>(q + (row * H + j) * kHeadDim)[c];
-    float* d = qs + j * kQStride + c * 8;
-    reinterpret_cast<float4*>(d)[0] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-    reinterpret_cast<float4*>(d)[1] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+  // the partial last block of this prefix: mean of keys Mfull*B .. P-1 (fp32)
+  if (has_part) {
+    const int s0 = Mfull * B, cnt = P - s0;
+    const uint16_t* kr = k + ((int64_t)n * L + s0) * kHeadDim + tid;
+    float a = 0.f;
+    for (int s = 0; s < cnt; ++s) a += bf16_to_f32(kr[(int64_t)s * kHeadDim]);
+    kpart[tid] = a / (float)cnt;
   }
-  // pooled keys of the chunk's full blocks; unused slots are zero
-  for (int e = tid; e < kCh * (kHeadDim / 4); e += kRouteThreads) {
+  // stage q rows (16-byte copies) and the chunk's pooled keys as bf16 hi/lo; every load
+  // of a thread is issued before any is stored
+  constexpr int kQPer = 16 * 4 * MT * (kHeadDim / 8) / kRouteThreads;
+  constexpr int kKPer = kCh * (kHeadDim / 4) / kRouteThreads;
+  uint4 qv[kQPer];
+  float4 kv[kKPer];
+#pragma unroll
+  for (int i = 0; i < kQPer; ++i) {
+    const int e = tid + i * kRouteThreads;
+    const int j = e / (kHeadDim / 8), c = e % (kHeadDim / 8);
+    qv[i] = j < H ? reinterpret_cast<const uint4*>(q + (row * H + j) * kHeadDim)[c]
+                  : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < kKPer; ++i) {
+    const int e = tid + i * kRouteThreads;
     const int bb = e / (kHeadDim / 4), c = e % (kHeadDim / 4);
     const int b = b0 + bb;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (bb < nb && b < Mfull)
-      v = reinterpret_cast<const float4*>(k_pool + ((int64_t)n * Mpool + b) * kHeadDim)[c];
-    reinterpret_cast<float4*>(kp + bb * kQStride)[c] = v;
+    kv[i] = (bb < nb && b < Mfull)
+                ? reinterpret_cast<const float4*>(k_pool + ((int64_t)n * Mpool + b) * kHeadDim)[c]
+                : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < kQPer; ++i) {
+    const int e = tid + i * kRouteThreads;
+    const int j = e / (kHeadDim / 8), c = e % (kHeadDim / 8);
+    *reinterpret_cast<uint4*>(qs + j * kRowPad + c * 8) = qv[i];
+  }
+  __syncthreads();   // kpart complete
+#pragma unroll
+  for (int i = 0; i < kKPer; ++i) {
+    const int e = tid + i * kRouteThreads;
+    const int bb = e / (kHeadDim / 4), c = e % (kHeadDim / 4);
+    float4 v = kv[i];
+    if (has_part && bb == Mfull - b0) v = reinterpret_cast<const float4*>(kpart)[c];
+    const float hx = __bfloat162float(__float2bfloat16_rn(v.x));
+    const float hy = __bfloat162float(__float2bfloat16_rn(v.y));
+    const float hz = __bfloat162float(__float2bfloat16_rn(v.z));
+    const float hw = __bfloat162float(__float2bfloat16_rn(v.w));
+    uint2 hi, lo;
+    hi.x = pack_bf16(hx, hy);
+    hi.y = pack_bf16(hz, hw);
+    lo.x = pack_bf16(v.x - hx, v.y - hy);
+    lo.y = pack_bf16(v.z - hz, v.w - hw);
+    *reinterpret_cast<uint2*>(khi + bb * kRowPad + c * 4) = hi;
+    *reinterpret_cast<uint2*>(klo + bb * kRowPad + c * 4) = lo;
   }
   __syncthreads();
-  // the partial last block of this prefix: mean of keys Mfull*B .. P-1
-  if (Mfull < M && Mfull >= b0 && Mfull < b0 + nb) {
-    const int s0 = Mfull * B, cnt = P - s0;
-    const int dim = tid % kHeadDim, part = tid / kHeadDim;   // 2 parts
-    float a = 0.f;
-    const uint16_t* kr = k + ((int64_t)n * L + s0) * kHeadDim + dim;
-    for (int s = part; s < cnt; s += kRouteThreads / kHeadDim) a += bf16_to_f32(kr[(int64_t)s * kHeadDim]);
-    float* tmp = ev;   // 128 floats of scratch
-    if (part == 1) tmp[dim] = a;
-    __syncthreads();
-    if (part == 0) kp[(Mfull - b0) * kQStride + dim] = (a + tmp[dim]) / (float)cnt;
-    __syncthreads();
-  }
 
-  const int hp = tid & 31, bq = tid >> 5;   // bq: 8 groups of 4 blocks
-  float acc[HG][4];
+  // S = Q K^T on the tensor cores; thread (g = lane/4, c = lane%4) holds rows g, g+8 and
+  // columns 2c, 2c+1 of every 16 x 8 tile
+  const int g = lane >> 2, c4 = lane & 3;
+  constexpr int kNT = kCh / 8;
+  float acc[MT][kNT][4];
 #pragma unroll
-  for (int m = 0; m < HG; ++m)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
-#pragma unroll 4
-  for (int d = 0; d < kHeadDim; d += 4) {
-    float4 qv[HG], kv[4];
+    for (int t = 0; t < kNT; ++t)
 #pragma unroll
-    for (int m = 0; m < HG; ++m) qv[m] = *reinterpret_cast<const float4*>(qs + (hp + 32 * m) * kQStride + d);
+      for (int i = 0; i < 4; ++i) acc[m][t][i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) kv[i] = *reinterpret_cast<const float4*>(kp + (4 * bq + i) * kQStride + d);
+  for (int k0 = 0; k0 < kHeadDim; k0 += 16) {
+    uint32_t bh[kNT][2], bl[kNT][2];
 #pragma unroll
-    for (int m = 0; m < HG; ++m)
+    for (int t = 0; t < kNT; ++t) {
+      const uint16_t* ph = khi + (t * 8 + g) * kRowPad + k0 + 2 * c4;
+      const uint16_t* pl = klo + (t * 8 + g) * kRowPad + k0 + 2 * c4;
+      bh[t][0] = *reinterpret_cast<const uint32_t*>(ph);
+      bh[t][1] = *reinterpret_cast<const uint32_t*>(ph + 8);
+      bl[t][0] = *reinterpret_cast<const uint32_t*>(pl);
+      bl[t][1] = *reinterpret_cast<const uint32_t*>(pl + 8);
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float x = acc[m][i];
-        x = fmaf(qv[m].x, kv[i].x, x); x = fmaf(qv[m].y, kv[i].y, x);
-        x = fmaf(qv[m].z, kv[i].z, x); x = fmaf(qv[m].w, kv[i].w, x);
-        acc[m][i] = x;
+    for (int m = 0; m < MT; ++m) {
+      const int r0 = (warp + 4 * m) * 16;
+      const uint16_t* pa = qs + (r0 + g) * kRowPad + k0 + 2 * c4;
+      uint32_t a[4];
+      a[0] = *reinterpret_cast<const uint32_t*>(pa);
+      a[1] = *reinterpret_cast<const uint32_t*>(pa + 8 * kRowPad);
+      a[2] = *reinterpret_cast<const uint32_t*>(pa + 8);
+      a[3] = *reinterpret_cast<const uint32_t*>(pa + 8 * kRowPad + 8);
+#pragma unroll
+      for (int t = 0; t < kNT; ++t) {
+        mma_bf16_16816(acc[m][t], a, bh[t][0], bh[t][1]);
+        mma_bf16_16816(acc[m][t], a, bl[t][0], bl[t][1]);
       }
+    }
   }
-  // sum_b ReLU(q_j . kp_b) over this thread's blocks, then over the 8 block groups
+  // sum_b ReLU(q_j . kp_b) over the chunk's valid blocks, per head
 #pragma unroll
-  for (int m = 0; m < HG; ++m) {
-    float sum = 0.f;
+  for (int m = 0; m < MT; ++m) {
+    float s_lo = 0.f, s_hi = 0.f;   // rows g and g + 8
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (4 * bq + i < nb) sum += fmaxf(acc[m][i], 0.f);
-    red[bq][hp + 32 * m] = sum;
+    for (int t = 0; t < kNT; ++t)
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (t * 8 + 2 * c4 + i < nb) {
+          s_lo += fmaxf(acc[m][t][i], 0.f);
+          s_hi += fmaxf(acc[m][t][2 + i], 0.f);
+        }
+    s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 1);
+    s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 2);
+    s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 1);
+    s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 2);
+    const int r0 = (warp + 4 * m) * 16;
+    if (c4 == 0) {
+      if (r0 + g < H) rsum[r0 + g] = s_lo;
+      if (r0 + g + 8 < H) rsum[r0 + g + 8] = s_hi;
+    }
   }
   __syncthreads();
-  if (tid < H) {
-    float sum = 0.f;
-#pragma unroll
-    for (int g = 0; g < kRouteThreads / 32; ++g) sum += red[g][tid];
-    partial[(row * nchunk + chunk) * H + tid] = sum;
-    __threadfence();
-  }
+  for (int j = tid; j < H; j += kRouteThreads) partial[(row * nchunk + chunk) * H + j] = rsum[j];
+  __threadfence();
   __syncthreads();
   const int nch = (M + kCh - 1) / kCh;
   if (tid == 0) s_last = atomicAdd(&counters[row], 1) == nch - 1;
@@ -196,20 +270,20 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   if (tid < 32) select_top_h(ev, H, h, heads + row * h);
 }
 
-template <int HG>
-static cudaError_t launch_hg(const uint16_t* q, const float* w, const uint16_t* k,
+template <int MT>
+static cudaError_t launch_mt(const uint16_t* q, const float* w, const uint16_t* k,
                              const float* k_pool, const int32_t* pos, int rows, int T, int H,
                              int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
                              int nchunk, int* counters, int* status, cudaStream_t st) {
   const int Mpool = (int)((L + B - 1) / B);
-  const size_t smem = (size_t)(32 * HG + kCh) * kQStride * sizeof(float);
-  cudaError_t err = cudaFuncSetAttribute(route_kernel<HG>,
+  const size_t smem = (size_t)(16 * 4 * MT + 2 * kCh) * kRowPad * sizeof(uint16_t);
+  cudaError_t err = cudaFuncSetAttribute(route_kernel<MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
     dim3 grid(nchunk, (unsigned)nr);
-    route_kernel<HG><<<grid, kRouteThreads, smem, st>>>(q, k, k_pool, pos, T, H, L, B, Mpool,
+    route_kernel<MT><<<grid, kRouteThreads, smem, st>>>(q, k, k_pool, pos, T, H, L, B, Mpool,
                                                         partial, nchunk, status, row0, w, h,
                                                         counters, heads, E);
     err = cudaGetLastError();
@@ -227,12 +301,11 @@ cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
   const int rows = nseq * T;
   cudaError_t err = cudaMemsetAsync(counters, 0, (size_t)rows * sizeof(int), st);
   if (err != cudaSuccess) return err;
-  switch ((H + 31) / 32) {
-    case 1: return launch_hg<1>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk, counters, status, st);
-    case 2: return launch_hg<2>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk, counters, status, st);
-    case 3: return launch_hg<3>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk, counters, status, st);
-    default: return launch_hg<4>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk, counters, status, st);
-  }
+  if (H <= 64)
+    return launch_mt<1>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk,
+                        counters, status, st);
+  return launch_mt<2>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk,
+                      counters, status, st);
 }
 
 }  // namespace misa

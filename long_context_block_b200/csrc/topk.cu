@@ -684,7 +684,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   __shared__ __align__(16) uint32_t hist[kSubBucketWords];     // histogram, then buckets
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t red[2];
-  __shared__ uint32_t s_cut, s_total, s_big, s_fill, s_flag, s_digit, s_above, s_top, s_nsub;
+  __shared__ uint32_t s_cut, s_total, s_big, s_flag, s_digit, s_above, s_top, s_nsub;
   __shared__ __align__(8) uint64_t lbar;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t row = row0 + blockIdx.x;
@@ -712,7 +712,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   if (t < 4 && h0 + nbulk + t < n) keys[h0 + nbulk + t] = __float_as_uint(x[h0 + nbulk + t]);
   for (int b = t; b < kScoreHistBins; b += NT) hist[b] = (ghist && n > (int)target)
                                                     ? ghist[row * kScoreHistBins + b] : 0u;
-  if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; s_fill = 0; s_top = 0; }
+  if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; s_top = 0; }
   if (nbulk > 0) {   // bounded wait for the copy; on expiry the row's result is void
     long long t0 = clock64();
     bool landed = true;
@@ -764,16 +764,31 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   }
   __syncthreads();
   const bool fits = C <= (uint32_t)CAP;
+  // Candidates carry their position e in the row; the index map (if any) is applied to
+  // the k outputs only.  Warp w compacts the contiguous slice [w0, w1) of the row in
+  // 32-key steps: a counting pass, one block scan over the warps, then ballot ranks.
+  constexpr int kWarps = NT / 32;
+  const int wper = (((n + kWarps - 1) / kWarps) + 31) & ~31;
+  const int w0 = min(warp * wper, n), w1 = min(w0 + wper, n);
+  const uint32_t below = (1u << lane) - 1u;
   if (fits) {
-    for (int base = 0; base < n; base += NT) {
-      const int e = base + t;
-      const uint32_t key = e < n ? keys[e] : 0u;
-      const bool take = e < n && (key >> (32 - kScoreHistBits)) >= cut;
+    const uint32_t kcut = cut << (32 - kScoreHistBits);   // keys >= kcut are candidates
+    uint32_t cnt = 0;
+#pragma unroll 4
+    for (int e = w0 + lane; e < w1; e += 32) cnt += keys[e] >= kcut ? 1u : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    uint32_t tot;
+    uint32_t p = __shfl_sync(0xffffffffu,
+                             block_excl_scan_nt<NT>(lane == 0 ? cnt : 0u, warp_sums, tot), 0);
+#pragma unroll 4
+    for (int e0 = w0; e0 < w1; e0 += 32) {
+      const int e = e0 + lane;
+      const uint32_t key = e < w1 ? keys[e] : 0u;
+      const bool take = e < w1 && key >= kcut;
       const uint32_t m = __ballot_sync(0xffffffffu, take);
-      uint32_t wb = 0;
-      if (lane == 0 && m) wb = atomicAdd(&s_fill, (uint32_t)__popc(m));
-      wb = __shfl_sync(0xffffffffu, wb, 0);
-      if (take) cand[wb + __popc(m & ((1u << lane) - 1u))] = compose(key, imap ? imap[e] : e);
+      if (take) cand[p + __popc(m & below)] = compose(key, e);
+      p += __popc(m);
     }
   } else {
     // crowded cutoff bin: exact threshold by a radix select over the resident keys, then
@@ -815,12 +830,8 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       __syncthreads();
     }
     const uint32_t thr = prefix;
-    // Warp w compacts the contiguous slice [w0, w1) of the row in 32-key steps, so that
-    // ranks in (warp, step, lane) order are ranks in index order: one block scan places
+    // Ranks in (warp, step, lane) order are ranks in index order: one block scan places
     // every warp's keys above the threshold and its equal ones.
-    constexpr int kWarps = NT / 32;
-    const int wper = (((n + kWarps - 1) / kWarps) + 31) & ~31;
-    const int w0 = min(warp * wper, n), w1 = min(w0 + wper, n);
     uint32_t ngt = 0, neq = 0;
     for (int e = w0 + lane; e < w1; e += 32) {
       const uint32_t key = keys[e];
@@ -844,11 +855,10 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       const bool eq = e < w1 && key == thr;
       const uint32_t mg = __ballot_sync(0xffffffffu, gt);
       const uint32_t me = __ballot_sync(0xffffffffu, eq);
-      const uint32_t below = (1u << lane) - 1u;
-      if (gt) cand[gpos + __popc(mg & below)] = compose(key, imap ? imap[e] : e);
+      if (gt) cand[gpos + __popc(mg & below)] = compose(key, e);
       if (eq) {
         const uint32_t r = epos + __popc(me & below);
-        if (r < kneed) cand[G + r] = compose(key, imap ? imap[e] : e);
+        if (r < kneed) cand[G + r] = compose(key, e);
       }
       gpos += __popc(mg);
       epos += __popc(me);
@@ -877,7 +887,8 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     const int64_t o = row * topk + i;
     if ((uint32_t)i < target) {
       const uint64_t v = sorted[i];
-      idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
+      const int32_t e = (int32_t)(~(uint32_t)(v & 0xffffffffu));   // position in the row
+      idx[o] = imap ? imap[e] : e;
       if (vals) vals[o] = key_score((uint32_t)(v >> 32));
     } else {
       idx[o] = -1;

@@ -713,6 +713,29 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   for (int b = t; b < kScoreHistBins; b += NT) hist[b] = (ghist && n > (int)target)
                                                     ? ghist[row * kScoreHistBins + b] : 0u;
   if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; s_top = 0; }
+  // Warp w owns the contiguous slice [w0, w1) of the row, walked in 32-key steps, in every
+  // pass below; the candidates carry their position e in the row, and the index map (if
+  // any) is applied to the k outputs only.
+  constexpr int kWarps = NT / 32;
+  const int wper = (((n + kWarps - 1) / kWarps) + 31) & ~31;
+  const int w0 = min(warp * wper, n), w1 = min(w0 + wper, n);
+  const uint32_t below = (1u << lane) - 1u;
+  uint32_t cut = 0, btop = 0, C = 0;
+  const bool select = (uint32_t)n > target;      // else every score is selected
+  const bool given = ghist != nullptr && select;   // cutoff known before the keys arrive
+  if (given) {   // runs while the bulk copy is in flight
+    __syncthreads();
+    HistView<NT> hv;
+    cut = hist_cutoff<NT>(hist, target, hv, warp_sums, s_cut, s_total, s_big);
+    uint32_t top = 0;
+#pragma unroll
+    for (int i = HistView<NT>::kPer - 1; i >= 0; --i)
+      if (hv.c[i]) top = max(top, (uint32_t)(hv.hi - 1 - i));
+    if (top) atomicMax(&s_top, top);
+    __syncthreads();
+    btop = s_top;
+    C = s_total;
+  }
   if (nbulk > 0) {   // bounded wait for the copy; on expiry the row's result is void
     long long t0 = clock64();
     bool landed = true;
@@ -730,26 +753,32 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     }
   }
   __syncthreads();
-  for (int e = t; e < n; e += NT) keys[e] = score_key(__uint_as_float(keys[e]));
-  __syncthreads();
-  uint32_t cut, btop, C;
-  if ((uint32_t)n <= target) {
-    // every score is selected
-    uint32_t lo = 0xffffffffu, hi = 0;
-    for (int e = t; e < n; e += NT) {
-      const uint32_t b = keys[e] >> (32 - kScoreHistBits);
+  // scores -> keys, and in the same pass: the histogram (none given), the bin range (all
+  // selected) or this warp's candidate count (cutoff given)
+  const uint32_t kgiven = cut << (32 - kScoreHistBits);
+  uint32_t lo = 0xffffffffu, hi = 0, cnt = 0;
+#pragma unroll 4
+  for (int e = w0 + lane; e < w1; e += 32) {
+    const uint32_t kk = score_key(__uint_as_float(keys[e]));
+    keys[e] = kk;
+    const uint32_t b = kk >> (32 - kScoreHistBits);
+    if (!select) {
       lo = min(lo, b);
       hi = max(hi, b);
+    } else if (given) {
+      cnt += kk >= kgiven ? 1u : 0u;
+    } else {
+      atomicAdd(&hist[b], 1u);
     }
+  }
+  __syncthreads();
+  if (!select) {
     block_minmax<NT>(lo, hi, red);
     cut = lo;
     btop = hi;
     C = (uint32_t)n;
-  } else {
-    if (!ghist) {
-      for (int e = t; e < n; e += NT) atomicAdd(&hist[keys[e] >> (32 - kScoreHistBits)], 1u);
-      __syncthreads();
-    }
+    cnt = (uint32_t)(w1 - w0) / 32u + ((uint32_t)lane < (uint32_t)((w1 - w0) & 31) ? 1u : 0u);
+  } else if (!given) {
     HistView<NT> hv;
     cut = hist_cutoff<NT>(hist, target, hv, warp_sums, s_cut, s_total, s_big);
     // highest occupied bin
@@ -764,31 +793,28 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   }
   __syncthreads();
   const bool fits = C <= (uint32_t)CAP;
-  // Candidates carry their position e in the row; the index map (if any) is applied to
-  // the k outputs only.  Warp w compacts the contiguous slice [w0, w1) of the row in
-  // 32-key steps: a counting pass, one block scan over the warps, then ballot ranks.
-  constexpr int kWarps = NT / 32;
-  const int wper = (((n + kWarps - 1) / kWarps) + 31) & ~31;
-  const int w0 = min(warp * wper, n), w1 = min(w0 + wper, n);
-  const uint32_t below = (1u << lane) - 1u;
   if (fits) {
     const uint32_t kcut = cut << (32 - kScoreHistBits);   // keys >= kcut are candidates
-    uint32_t cnt = 0;
+    if (select && !given) {   // count this lane's candidates (counted above otherwise)
+      cnt = 0;
 #pragma unroll 4
-    for (int e = w0 + lane; e < w1; e += 32) cnt += keys[e] >= kcut ? 1u : 0u;
+      for (int e = w0 + lane; e < w1; e += 32) cnt += keys[e] >= kcut ? 1u : 0u;
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     uint32_t tot;
     uint32_t p = __shfl_sync(0xffffffffu,
                              block_excl_scan_nt<NT>(lane == 0 ? cnt : 0u, warp_sums, tot), 0);
+    C = min(tot, (uint32_t)CAP);
 #pragma unroll 4
     for (int e0 = w0; e0 < w1; e0 += 32) {
       const int e = e0 + lane;
       const uint32_t key = e < w1 ? keys[e] : 0u;
       const bool take = e < w1 && key >= kcut;
       const uint32_t m = __ballot_sync(0xffffffffu, take);
-      if (take) cand[p + __popc(m & below)] = compose(key, e);
-      p += __popc(m);
+      const uint32_t r = p + __popc(m & below);
+      if (take && r < (uint32_t)CAP) cand[r] = compose(key, e);   // (a histogram that
+      p += __popc(m);                                            //  disagrees cannot overflow)
     }
   } else {
     // crowded cutoff bin: exact threshold by a radix select over the resident keys, then
@@ -883,16 +909,31 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     __syncthreads();
     row_bitonic<NT, RC::kEMax>(sorted, sortn);
   }
-  for (int i = t; i < topk; i += NT) {
-    const int64_t o = row * topk + i;
-    if ((uint32_t)i < target) {
-      const uint64_t v = sorted[i];
-      const int32_t e = (int32_t)(~(uint32_t)(v & 0xffffffffu));   // position in the row
-      idx[o] = imap ? imap[e] : e;
-      if (vals) vals[o] = key_score((uint32_t)(v >> 32));
-    } else {
-      idx[o] = -1;
-      if (vals) vals[o] = __int_as_float(0xff800000);
+  // outputs, four per thread per step so that the index-map loads overlap
+  for (int i0 = t; i0 < topk; i0 += 4 * NT) {
+    int32_t id[4];
+    uint32_t key[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * NT;
+      id[u] = -1;
+      key[u] = 0u;
+      if (i < topk && (uint32_t)i < target) {
+        const uint64_t v = sorted[i];
+        const int32_t e = (int32_t)(~(uint32_t)(v & 0xffffffffu));   // position in the row
+        id[u] = imap ? imap[e] : e;
+        key[u] = (uint32_t)(v >> 32);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * NT;
+      if (i < topk) {
+        const int64_t o = row * topk + i;
+        const bool ok = (uint32_t)i < target;
+        idx[o] = ok ? id[u] : -1;
+        if (vals) vals[o] = ok ? key_score(key[u]) : __int_as_float(0xff800000);
+      }
     }
   }
 }

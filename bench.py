@@ -116,21 +116,26 @@ class ClockSampler:
 
 
 def block_form(wl) -> bool:
-    """Whether the scorer shares key tiles among blocks of 256 / h queries (prefill)."""
-    hs = 8 if wl.h <= 8 else 16
-    return wl.T >= 256 // hs and wl.T >= 16
+    """Whether the scorer shares key tiles among the queries of a sequence (any T > 1)."""
+    return wl.T >= 2
 
 
 def misa_step_launches(wl) -> int:
     """Kernels one MISA step launches, following the library's dispatch: pooling, the router
-    (one kernel on CUDA cores, or four on tensor cores for many queries per sequence), the
-    scorer's gather/offsets kernel and the scorer, then the top-k (histogram path for long
-    decode rows: two kernels, three above k = 4096; otherwise one)."""
-    n = 1 + (4 if (128 % wl.H == 0 and wl.T >= 4 * (128 // wl.H) and -(-wl.L // wl.B) <= 256)
-             else 1)
+    (one kernel, or four on tcgen05 for many queries per sequence), the scorer's
+    gather/offsets kernel and the scorer, then the top-k: one kernel, except decode rows
+    longer than 40960 scores (or k > 3072) with the scorer's histogram, which take a
+    scatter and a group kernel (and an overflow kernel above k = 4096)."""
+    qt = 128 // wl.H if 128 % wl.H == 0 else 0
+    route_tc = (qt > 0 and wl.T >= 4 * qt and -(-wl.L // wl.B) <= 256
+                and (wl.nseq == 1 or wl.T % qt == 0))
+    n = 1 + (4 if route_tc else 1)
     n += 2
     hist_path = wl.rows <= 1024 and wl.L >= 8192 and not block_form(wl)
-    n += (2 + (wl.topk > 4096)) if hist_path else 1
+    if hist_path and not (wl.L <= 40960 and wl.topk <= 3072):
+        n += 2 + (wl.topk > 4096)
+    else:
+        n += 1
     return n
 
 
@@ -384,22 +389,26 @@ def run_cuda(args, wl):
     if os.path.exists(tfile):
         with open(tfile) as f:
             traffic = json.load(f).get(wl.name, {}).get("score_tc_kernel")
-    if block_form(wl):
-        flops = algorithmic_flops_score(wl)
+    # the kernel's bound is whichever of its algorithmic flops and bytes takes longer at peak
+    flops = algorithmic_flops_score(wl)
+    score_bytes = algorithmic_bytes_score(wl)
+    form = "block form" if block_form(wl) else "decode form"
+    if flops / (peaks["bf16"] * 1e12) > score_bytes / (peaks["hbm"] * 1e9):
         achieved = flops / (ms_score_kernel * 1e-3) / 1e12
-        roofline = {"kernel": "score_tc_kernel (routed scoring, block form)", "bound": "tensor",
+        roofline = {"kernel": f"score_tc_kernel (routed scoring, {form})", "bound": "tensor",
                     "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
                     "frac": achieved / peaks["bf16"], "traffic": traffic,
                     "peak_source": peaks["source"] + " bf16 dense (burst)",
-                    "algorithmic_flops": flops, "avg_ms": ms_score_kernel}
+                    "algorithmic_flops": flops, "algorithmic_bytes": score_bytes,
+                    "avg_ms": ms_score_kernel}
     else:
-        score_bytes = algorithmic_bytes_score(wl)
         achieved = score_bytes / (ms_score_kernel * 1e-3) / 1e9
-        roofline = {"kernel": "score_tc_kernel (routed scoring, decode form)", "bound": "hbm",
+        roofline = {"kernel": f"score_tc_kernel (routed scoring, {form})", "bound": "hbm",
                     "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm"], "traffic": traffic,
                     "peak_source": peaks["source"] + " HBM copy",
-                    "algorithmic_bytes": score_bytes, "avg_ms": ms_score_kernel}
+                    "algorithmic_bytes": score_bytes, "algorithmic_flops": flops,
+                    "avg_ms": ms_score_kernel}
 
     launches_per_step = misa_step_launches(wl)
     if ms_kept is not None:

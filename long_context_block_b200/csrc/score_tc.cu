@@ -13,8 +13,10 @@
 // (query, key) score leaves the SM once, as fp32.
 //   * decode form (QB = 1): every row streams its own prefix; the contraction is
 //     HBM-bound (256 bytes of keys per token), N = HS <= 128.
-//   * block form (QB = 256 / HS): QB queries share every key tile, N = 256; the
-//     contraction is tensor-bound (prefill), 2 * 128 * 256 * 128 flops per tile.
+//   * block form (QB > 1): QB queries of a sequence share every key tile.  With
+//     QB = 256 / HS (prefill) N = 256 and the contraction is tensor-bound, 2 * 128 *
+//     256 * 128 flops per tile; a few queries (multi-token decode) take a narrower
+//     block (N >= 32) and read each key once per sequence instead of once per query.
 //
 // Warp roles: warp 0 TMA producer (ring of 32 KB key tiles, each two 64-column boxes with
 // the 128-byte swizzle; per unit the q tile and its weights); warp 1 MMA issuer (one
@@ -615,13 +617,18 @@ struct Plan {
 
 Plan plan_for(int nh, int T, bool gather = false) {
   Plan p;
-  // block form when a sequence has enough queries to fill a 256-column B operand (rows
-  // with their own token lists always take the decode form)
+  // Block form whenever a sequence has several queries: QB of them share every key tile.
+  // Full width (N = 256) from 256 / HS queries on (prefill); a few queries (multi-token
+  // decode) take the next power of two >= T, at least 32 columns, so each unit still reads
+  // the sequence's keys once.  Rows with their own token lists take the decode form.
   const int hs_pow2 = nh <= 8 ? 8 : nh <= 16 ? 16 : nh <= 32 ? 32 : nh <= 64 ? 64 : 128;
   const int qb = 256 / hs_pow2;
-  if (!gather && T >= qb && T >= 16) {
+  if (!gather && T >= 2) {
+    int q = 2;
+    while (q < T && q < qb) q <<= 1;
+    while (q * hs_pow2 < 32) q <<= 1;
     p.HS = hs_pow2;
-    p.QB = qb;
+    p.QB = q;
   } else {
     p.HS = ((nh + 15) / 16) * 16;
     p.QB = 1;
@@ -705,9 +712,18 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
   MISA_TC_CASE(96, 1)
   MISA_TC_CASE(112, 1)
   MISA_TC_CASE(128, 1)
+  MISA_TC_CASE(8, 4)
+  MISA_TC_CASE(8, 8)
+  MISA_TC_CASE(8, 16)
   MISA_TC_CASE(8, 32)
+  MISA_TC_CASE(16, 2)
+  MISA_TC_CASE(16, 4)
+  MISA_TC_CASE(16, 8)
   MISA_TC_CASE(16, 16)
+  MISA_TC_CASE(32, 2)
+  MISA_TC_CASE(32, 4)
   MISA_TC_CASE(32, 8)
+  MISA_TC_CASE(64, 2)
   MISA_TC_CASE(64, 4)
   MISA_TC_CASE(128, 2)
 #undef MISA_TC_CASE

@@ -87,6 +87,15 @@ WORKLOADS = {
     "glm5_decode_128k": Workload("glm5_decode_128k", nseq=8, T=1, L=131072, H=32, d=128,
                                  h=8, B=128, topk=2048, kprime=8192, pos_mode="tail",
                                  drift=True, needles=8),
+    # multi-token decode (several draft positions per step): 32 sequences x 4 queries at
+    # the last 4 positions of a 32K prefix
+    "dsv32_mtp_32k": Workload("dsv32_mtp_32k", nseq=32, T=4, L=32768, H=64, d=128, h=8,
+                              B=64, topk=2048, kprime=8192, pos_mode="tail", drift=True,
+                              needles=8),
+    # 16 queries per sequence over a 32K prefix (a speculative draft of 16 positions)
+    "dsv32_draft16_32k": Workload("dsv32_draft16_32k", nseq=32, T=16, L=32768, H=64, d=128,
+                                  h=8, B=64, topk=2048, kprime=8192, pos_mode="tail",
+                                  drift=True, needles=8),
     # MISA-dagger re-rank against dense DSA at 128K: 16 sequences x 1 query, k' = 8192
     "dagger_128k": Workload("dagger_128k", nseq=16, T=1, L=131072, H=64, d=128, h=8,
                             B=64, topk=2048, kprime=8192, pos_mode="tail", drift=True,

@@ -45,7 +45,8 @@ def test_workspace_sizes(lib):
     hp = lambda rows: a256(rows * 4096 * 4) + a256(rows * 16 * 4) + a256(rows * 16 * 4096 * 8)
     assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 16) + hp(32)
     assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 64) + hp(32)
-    assert ws(2, 1, 16, 64, 128, 2048, 64, 8, 256, 512) == 256 + 16 * 2048 * 4 + tc(16, 16)
+    # 16 queries of one sequence share key tiles: one unit of 16 queries x 8 slots
+    assert ws(2, 1, 16, 64, 128, 2048, 64, 8, 256, 512) == 256 + 16 * 2048 * 4 + tc(1, 128)
     # re-rank: sorted candidate ids, their scores, per-row counts, tensor-core scratch
     # (every row in the decode form with all 64 heads)
     assert ws(4, 16, 1, 64, 128, 131072, 64, 8, 2048, 8192) == \

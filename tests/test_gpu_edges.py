@@ -50,6 +50,14 @@ CASES = {
     "max_topk": dict(nseq=1, T=2, L=20000, topk=16384, kprime=16384, B=128),
     # re-rank over more candidates than the row top-k keeps resident (16384 > 8192)
     "dagger_wide_kprime": dict(nseq=1, T=2, L=20000, topk=2048, kprime=16384, B=128),
+    # one query per sequence: the decode form of the scorer
+    "decode_T1_ragged": dict(nseq=4, T=1, L=777, topk=64, kprime=128),
+    "decode_T1_H16_B1": dict(nseq=3, T=1, L=300, H=16, h=5, B=1, topk=32, kprime=64),
+    # a few queries per sequence (multi-token decode): narrow query blocks
+    "mtp_T2": dict(nseq=3, T=2, L=900, topk=64, kprime=128),
+    "mtp_T3_H16": dict(nseq=2, T=3, L=1500, H=16, h=4, topk=100, kprime=200),
+    "mtp_T4_H64": dict(nseq=2, T=4, L=2000, H=64, h=8, topk=128, kprime=256),
+    "mtp_T9_H32": dict(nseq=2, T=9, L=1200, H=32, h=8, topk=64, kprime=128),
     # many queries per sequence: tensor-core router and query-block scorer
     "blocks_two_seqs_H16": dict(nseq=2, T=64, L=1000, H=16, h=4, topk=64, kprime=128),
     "blocks_H64_B32": dict(nseq=1, T=40, L=3000, H=64, h=8, B=32, topk=128, kprime=256),

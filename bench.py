@@ -357,6 +357,24 @@ def run_cuda(args, wl):
     ms_dsa = timed(dsa_step, args.steps, args.warmup)
     decode = T == 1 and bool(np.all(x.pos == wl.L - 1))
     ms_kept = timed(kept_pool_step, args.steps, args.warmup) if decode else None
+
+    # selection agreement with dense DSA on the same inputs (outside the timed regions): the
+    # fraction of DSA's k tokens that MISA and MISA-dagger also select, averaged over rows
+    misa_step(0)
+    dsa_step(0)
+    dagger_step(0)
+    torch.cuda.synchronize()
+
+    def recall(sel, ref):
+        r = ref.reshape(-1, ref.shape[-1]).long()
+        s_ = sel.reshape(-1, sel.shape[-1]).long()
+        mask = torch.zeros((r.shape[0], wl.L + 1), dtype=torch.bool, device=dev)
+        mask.scatter_(1, torch.where(r >= 0, r, wl.L), True)
+        hit = mask.gather(1, torch.where(s_ >= 0, s_, wl.L)) & (s_ >= 0)
+        n_ref = (r >= 0).sum(1).clamp(min=1)
+        return float((hit.sum(1).float() / n_ref.float()).mean().item())
+
+    recalls = {"misa": recall(idx, didx), "misa_dagger": recall(gidx, didx)}
     # the routed scoring kernel alone (misa_score_rows: the scorer of misa_score_topk with the
     # same launch configuration), on the heads the MISA steps routed
     score_buf = torch.empty((nseq, T, wl.L), dtype=torch.float32, device=dev)
@@ -435,6 +453,7 @@ def run_cuda(args, wl):
             "misa_dagger": {"value": units * world / (ms_dagger * 1e-3), "ms_per_step": ms_dagger},
             "speedup_misa_vs_dsa": ms_dsa / ms_misa,
             "speedup_dagger_vs_dsa": ms_dsa / ms_dagger,
+            "recall_vs_dsa": recalls,
         },
         "e2e": {"value": units * world / (ms_e2e * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -23,35 +23,60 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4& v) {
   a[6] += bf16lo(v.w); a[7] += bf16hi(v.w);
 }
 
-// Blocks b0 .. b0 + Mu - 1 of every sequence (M blocks per sequence in `out`).
+// Blocks b0 .. b0 + Mu - 1 of every sequence (M blocks per sequence in `out`).  W warps
+// share one block: W = 1 for short blocks (a warp per block), W = 8 for long ones, whose
+// tokens the CTA's warps split before a shared-memory reduction.
+template <int W>
 __global__ void __launch_bounds__(256) pool_mean_kernel(const uint4* __restrict__ k, int nseq,
                                                         int64_t L, int B, int M, int b0, int Mu,
                                                         float* __restrict__ out) {
+  __shared__ float red[W > 1 ? W : 1][kHeadDim];
   const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int half = lane >> 4;   // 0: even tokens of the block, 1: odd tokens
+  const int wic = (threadIdx.x >> 5) % W;   // warp within its block's group
+  const int64_t team = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / (32 * W);
+  const int64_t nteams = ((int64_t)gridDim.x * blockDim.x) / (32 * W);
+  const int half = lane >> 4;   // 0: even tokens of the pair, 1: odd tokens
   const int vec = lane & 15;    // which 16-byte slice of the key row
   const int64_t items = (int64_t)nseq * Mu;
-  for (int64_t it = warp; it < items; it += nwarps) {
-    const int64_t n = it / Mu;
-    const int64_t b = b0 + (it - n * Mu);
-    const int64_t s0 = b * B;
-    const int64_t s1 = min(s0 + (int64_t)B, L);
-    const uint4* base = k + n * L * 16 + vec;   // a key row is 16 uint4
+  for (int64_t base_it = blockIdx.x * ((int64_t)blockDim.x / (32 * W)); base_it < items;
+       base_it += nteams) {
+    const int64_t it = base_it + (team - blockIdx.x * ((int64_t)blockDim.x / (32 * W)));
+    const bool live = it < items;
     float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int64_t s = s0 + half;
-    for (; s + 14 < s1; s += 16) {
-      uint4 v[8];
+    int64_t n = 0, b = 0, s0 = 0, s1 = 0;
+    if (live) {
+      n = it / Mu;
+      b = b0 + (it - n * Mu);
+      s0 = b * B;
+      s1 = min(s0 + (int64_t)B, L);
+      const uint4* base = k + n * L * 16 + vec;   // a key row is 16 uint4
+      const int64_t step = 2 * W;                 // tokens between this warp's pairs
+      int64_t s = s0 + 2 * wic + half;
+      for (; s + 7 * step < s1; s += 8 * step) {
+        uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcs(base + (s + 2 * u) * 16);
+        for (int u = 0; u < 8; ++u) v[u] = __ldcs(base + (s + u * step) * 16);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc8(a, v[u]);
+        for (int u = 0; u < 8; ++u) acc8(a, v[u]);
+      }
+      for (; s < s1; s += step) acc8(a, __ldcs(base + s * 16));
     }
-    for (; s < s1; s += 2) acc8(a, __ldcs(base + s * 16));
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] += __shfl_down_sync(0xffffffffu, a[i], 16);
-    if (half == 0) {
+    if constexpr (W > 1) {
+      if (half == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[wic][vec * 8 + i] = a[i];
+      }
+      __syncthreads();
+      if (wic == 0 && half == 0) {
+        for (int w2 = 1; w2 < W; ++w2)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] += red[w2][vec * 8 + i];
+      }
+      __syncthreads();
+    }
+    if (live && wic == 0 && half == 0) {
       const float inv = 1.0f / (float)(s1 - s0);
       float4* o = reinterpret_cast<float4*>(out + (n * M + b) * kHeadDim + vec * 8);
       o[0] = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
@@ -73,10 +98,16 @@ cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, floa
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (items + 7) / 8;           // 8 warps per CTA
-  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  pool_mean_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M, b0, Mu,
-                                         k_pool);
+  if (B >= 256) {   // a CTA of 8 warps per block
+    const int grid = (int)(items < (int64_t)sms * 8 ? items : (int64_t)sms * 8);
+    pool_mean_kernel<8><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M,
+                                              b0, Mu, k_pool);
+  } else {          // a warp per block
+    const int64_t want = (items + 7) / 8;
+    const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+    pool_mean_kernel<1><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M,
+                                              b0, Mu, k_pool);
+  }
   return cudaGetLastError();
 }
 

@@ -113,7 +113,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   if (b0 >= M) return;
   const int nb = min(b0 + kCh, M) - b0;
   const int64_t n = row / T;
-  const int HT = 16 * 4 * MT;   // head rows staged (zero past H)
   const bool has_part = Mfull < M && Mfull >= b0 && Mfull < b0 + nb;
 
   // the partial last block of this prefix: mean of keys Mfull*B .. P-1 (fp32)

@@ -221,13 +221,14 @@ def test_dagger_candidates_any_order_with_repeats(M):
             tl.check_scores(vals[n, t], d_ref[idx[n, t]], what=f"dagger vals {n},{t}")
 
 
-def test_pool_keys_range_refreshes_only_changed_blocks(M):
+@pytest.mark.parametrize("B", [64, 512])
+def test_pool_keys_range_refreshes_only_changed_blocks(M, B):
     """Eq. (4) kept up to date: after keys in a token range change, the refresh rewrites
     exactly the blocks meeting that range; the result equals a full re-pool bit for bit
-    (same kernel arithmetic) and the oracle's pooled keys within tolerance."""
+    (same kernel arithmetic) and the oracle's pooled keys within tolerance.  B = 512 takes
+    the form where a CTA's warps share one block."""
     import oracle.misa_oracle as orc
     from tests import tolerance as tl
-    B = 64
     wl = _wl(nseq=3, T=1, L=1000, B=B)
     x = make_inputs(wl, seed=17)
     _, _, k, _ = gpu_path.to_device(x)

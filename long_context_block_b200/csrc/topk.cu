@@ -36,6 +36,16 @@ __device__ __forceinline__ uint64_t compose(uint32_t key, int32_t id) {
   return ((uint64_t)key << 32) | (uint64_t)(~(uint32_t)id);
 }
 
+// Shared-histogram increment by a whole warp: lanes holding the same bin add once.  Used by
+// the exact (crowded-cutoff) passes, where a row's keys may all fall in one bin (exact zeros
+// from the ReLU, ties) and plain atomics would serialise on one address.  Every lane of the
+// warp must call it; `ok` = this lane has a key to count.
+__device__ __forceinline__ void warp_hist_add(uint32_t* h, uint32_t bin, bool ok) {
+  const uint32_t key = ok ? bin : 0xffffffffu;
+  const uint32_t m = __match_any_sync(0xffffffffu, key);
+  if (ok && (threadIdx.x & 31) == (uint32_t)(__ffs(m) - 1)) atomicAdd(&h[bin], (uint32_t)__popc(m));
+}
+
 // Block-wide exclusive prefix sum over one value per thread (all threads must call).
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums,
                                                     uint32_t& total) {
@@ -130,9 +140,10 @@ __device__ void select_row_global_nt(const float* __restrict__ x, const int32_t*
       const int nb = p == 2 ? 1024 : 2048;
       for (int b = tid; b < kBins; b += NT) hist[b] = 0;
       __syncthreads();
-      for (int i = tid; i < n; i += NT) {
-        const uint32_t key = score_key(x[i]);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+      for (int i0 = 0; i0 < n; i0 += NT) {   // block-wide steps (warp-wide histogram adds)
+        const int i = i0 + tid;
+        const uint32_t key = i < n ? score_key(x[i]) : 0u;
+        warp_hist_add(hist, (key >> shift) & (nb - 1), i < n && (key & mask) == prefix);
       }
       __syncthreads();
       // suffix scan: thread t covers bins nb-1-kPerT*t-i, i < kPerT
@@ -792,10 +803,35 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     C = s_total;
   }
   __syncthreads();
+  // A crowded cutoff bin (more candidates than CAP): refine the threshold with a histogram
+  // of the next 12 key bits of the keys in that bin, one more pass over the row; only rows
+  // with massive ties (exact zeros from the ReLU, equal keys) still overflow.
+  uint32_t kcut = cut << (32 - kScoreHistBits);   // keys >= kcut are candidates
+  bool refined = false;
+  if (select && C > (uint32_t)CAP) {
+    const uint32_t above = C - hist[cut];   // keys in the bins above the cutoff bin
+    __syncthreads();
+    for (int b = t; b < kScoreHistBins; b += NT) hist[b] = 0;
+    __syncthreads();
+#pragma unroll 4
+    for (int e = w0 + lane; e < w1; e += 32) {
+      const uint32_t kk = keys[e];
+      if ((kk >> (32 - kScoreHistBits)) == cut)
+        atomicAdd(&hist[(kk >> (32 - 2 * kScoreHistBits)) & (kScoreHistBins - 1)], 1u);
+    }
+    __syncthreads();
+    HistView<NT> hv2;
+    const uint32_t sc = hist_cutoff<NT>(hist, target - above, hv2, warp_sums, s_cut, s_total, s_big);
+    if (above + s_total <= (uint32_t)CAP) {
+      kcut |= sc << (32 - 2 * kScoreHistBits);
+      C = above + s_total;
+      refined = true;
+    }
+    __syncthreads();
+  }
   const bool fits = C <= (uint32_t)CAP;
   if (fits) {
-    const uint32_t kcut = cut << (32 - kScoreHistBits);   // keys >= kcut are candidates
-    if (select && !given) {   // count this lane's candidates (counted above otherwise)
+    if ((select && !given) || refined) {   // count this lane's candidates (else counted above)
       cnt = 0;
 #pragma unroll 4
       for (int e = w0 + lane; e < w1; e += 32) cnt += keys[e] >= kcut ? 1u : 0u;
@@ -825,9 +861,10 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       const int nb = p == 2 ? 1024 : 2048;
       for (int b = t; b < 2048; b += NT) hist[b] = 0;
       __syncthreads();
-      for (int e = t; e < n; e += NT) {
-        const uint32_t key = keys[e];
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+      for (int e0 = 0; e0 < n; e0 += NT) {   // block-wide steps (warp-wide histogram adds)
+        const int e = e0 + t;
+        const uint32_t key = e < n ? keys[e] : 0u;
+        warp_hist_add(hist, (key >> shift) & (nb - 1), e < n && (key & mask) == prefix);
       }
       __syncthreads();
       // suffix scan: thread t covers bins nb-1-kBinsPer*t-i, i < kBinsPer

@@ -29,6 +29,14 @@ __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float(u);
 }
 
+// First statements of a kernel started by launch_pdl: let the next kernel in the stream
+// begin launching, then wait until the previous kernel has completed and its writes are
+// visible (both are no-ops for a kernel launched without the attribute).
+__device__ __forceinline__ void pdl_prologue() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Record a device-side condition in the workspace status word (first one wins).
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);

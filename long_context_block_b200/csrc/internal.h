@@ -7,6 +7,26 @@
 
 namespace misa {
 
+// Launch with programmatic dependent launch allowed: the kernel may be scheduled while the
+// previous kernel in the stream finishes.  Every kernel launched this way starts with
+// pdl_prologue() (common.cuh), which waits for the previous kernel's completion and writes
+// before anything else, so stream order is kept.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Workspace layout helpers: every region starts on a 256-byte boundary.
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 

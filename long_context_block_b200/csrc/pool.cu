@@ -30,6 +30,7 @@ template <int W>
 __global__ void __launch_bounds__(256) pool_mean_kernel(const uint4* __restrict__ k, int nseq,
                                                         int64_t L, int B, int M, int b0, int Mu,
                                                         float* __restrict__ out) {
+  pdl_prologue();
   __shared__ float red[W > 1 ? W : 1][kHeadDim];
   const int lane = threadIdx.x & 31;
   const int wic = (threadIdx.x >> 5) % W;   // warp within its block's group
@@ -100,15 +101,14 @@ cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, floa
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (B >= 256) {   // a CTA of 8 warps per block
     const int grid = (int)(items < (int64_t)sms * 8 ? items : (int64_t)sms * 8);
-    pool_mean_kernel<8><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M,
-                                              b0, Mu, k_pool);
+    return launch_pdl(pool_mean_kernel<8>, dim3(grid), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(k), nseq, L, B, M, b0, Mu, k_pool);
   } else {          // a warp per block
     const int64_t want = (items + 7) / 8;
     const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-    pool_mean_kernel<1><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(k), nseq, L, B, M,
-                                              b0, Mu, k_pool);
+    return launch_pdl(pool_mean_kernel<1>, dim3(grid), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(k), nseq, L, B, M, b0, Mu, k_pool);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace misa

@@ -23,6 +23,7 @@ constexpr int kBitmapMaxBytes = 200 * 1024;
 __global__ void __launch_bounds__(kBitmapThreads) bitmap_candidates_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pos, int64_t L, int kprime,
     int32_t* __restrict__ sorted, int32_t* __restrict__ count, int* status, int64_t row0) {
+  pdl_prologue();
   extern __shared__ uint32_t bm[];   // [ceil(P / 32)] words
   __shared__ uint32_t warp_sums[kBitmapThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -126,12 +127,13 @@ cudaError_t launch_sort_candidates(const int32_t* cand, const int32_t* pos, int 
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
     if (bitmap)
-      bitmap_candidates_kernel<<<(unsigned)nr, kBitmapThreads, smem, st>>>(
-          cand, pos, L, kprime, sorted, count, status, row0);
-    else
+      e = launch_pdl(bitmap_candidates_kernel, dim3((unsigned)nr), dim3(kBitmapThreads), smem, st,
+                     cand, pos, L, kprime, sorted, count, status, row0);
+    else {
       sort_candidates_kernel<<<(unsigned)nr, kThreads, smem, st>>>(cand, pos, L, kprime, sortn,
                                                                    sorted, count, status, row0);
-    e = cudaGetLastError();
+      e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

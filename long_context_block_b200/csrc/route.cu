@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
     int64_t L, int B, int Mpool, float* __restrict__ partial, int nchunk, int* status,
     int64_t row0, const float* __restrict__ w, int h, int* __restrict__ counters,
     int32_t* __restrict__ heads, float* __restrict__ E) {
+  pdl_prologue();
   extern __shared__ __align__(16) uint16_t rsm[];
   uint16_t* qs = rsm;                                  // [16 * 4 * MT][kRowPad] bf16
   uint16_t* khi = qs + 16 * 4 * MT * kRowPad;          // [kCh][kRowPad]
@@ -282,10 +283,8 @@ static cudaError_t launch_mt(const uint16_t* q, const float* w, const uint16_t* 
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
     dim3 grid(nchunk, (unsigned)nr);
-    route_kernel<MT><<<grid, kRouteThreads, smem, st>>>(q, k, k_pool, pos, T, H, L, B, Mpool,
-                                                        partial, nchunk, status, row0, w, h,
-                                                        counters, heads, E);
-    err = cudaGetLastError();
+    err = launch_pdl(route_kernel<MT>, grid, dim3(kRouteThreads), smem, st, q, k, k_pool, pos, T,
+                     H, L, B, Mpool, partial, nchunk, status, row0, w, h, counters, heads, E);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     float* __restrict__ out, int64_t out_stride, int* status, uint32_t* __restrict__ hist,
     const int32_t* __restrict__ gidx, const int32_t* __restrict__ glen,
     const uint16_t* __restrict__ kraw) {
+  pdl_prologue();
   using C = Cfg<HS, QB>;
   constexpr int N = C::N;
   constexpr int kEpiThreads = 32 * C::kEpiWarps;
@@ -489,6 +490,7 @@ __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
     int hsel, int H, int HS, Units geo, const int32_t* __restrict__ pos, int units, int64_t L,
     const int32_t* __restrict__ glen, int gmax, uint4* __restrict__ qg, float* __restrict__ wg,
     int32_t* __restrict__ tile_off, int* status) {
+  pdl_prologue();
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   const int nh = heads ? hsel : H;
@@ -605,9 +607,9 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  score_tc_kernel<HS, QB, kGather><<<sms, C::kThreads, C::kSmemBytes, st>>>(
-      tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, status, hist, gidx, glen, kraw);
-  return cudaGetLastError();
+  return launch_pdl(score_tc_kernel<HS, QB, kGather>, dim3(sms), dim3(C::kThreads),
+                    (size_t)C::kSmemBytes, st, tk, tq, wg, pos, tile_off, units, geo, L, out,
+                    out_stride, status, hist, gidx, glen, kraw);
 }
 
 // Shape of the work units for nh heads and T queries per sequence.
@@ -677,9 +679,9 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
   int32_t* tile_off = reinterpret_cast<int32_t*>(c);
   if (p.QB > 1 || gather) hist = nullptr;
 
-  score_tc_prep_kernel<<<units, 1024, 0, st>>>(q, w, heads, hsel, H, p.HS, geo, pos, units, L,
-                                               glen, (int)out_stride, qg, wg, tile_off, status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(score_tc_prep_kernel, dim3(units), dim3(1024), 0, st, q, w, heads,
+                             hsel, H, p.HS, geo, pos, units, L, glen, (int)out_stride, qg, wg,
+                             tile_off, status);
   if (e != cudaSuccess) return e;
   CUtensorMap tk, tq;   // (the gather copies key rows with cp.async: tk goes unused)
   if (!make_map(&tk, k, (uint64_t)nseq * L, (uint32_t)kTileKeys) ||

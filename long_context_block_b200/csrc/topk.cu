@@ -37,8 +37,8 @@ __device__ __forceinline__ uint64_t compose(uint32_t key, int32_t id) {
 }
 
 // Shared-histogram increment by a whole warp: lanes holding the same bin add once.  Used by
-// the exact (crowded-cutoff) passes, where a row's keys may all fall in one bin (exact zeros
-// from the ReLU, ties) and plain atomics would serialise on one address.  Every lane of the
+// the row kernel's exact (crowded-cutoff) passes, where a row's keys may all fall in one bin
+// (exact zeros from the ReLU, ties) and plain atomics would serialise on one address.  Every lane of the
 // warp must call it; `ok` = this lane has a key to count.
 __device__ __forceinline__ void warp_hist_add(uint32_t* h, uint32_t bin, bool ok) {
   const uint32_t key = ok ? bin : 0xffffffffu;
@@ -140,10 +140,9 @@ __device__ void select_row_global_nt(const float* __restrict__ x, const int32_t*
       const int nb = p == 2 ? 1024 : 2048;
       for (int b = tid; b < kBins; b += NT) hist[b] = 0;
       __syncthreads();
-      for (int i0 = 0; i0 < n; i0 += NT) {   // block-wide steps (warp-wide histogram adds)
-        const int i = i0 + tid;
-        const uint32_t key = i < n ? score_key(x[i]) : 0u;
-        warp_hist_add(hist, (key >> shift) & (nb - 1), i < n && (key & mask) == prefix);
+      for (int i = tid; i < n; i += NT) {
+        const uint32_t key = score_key(x[i]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
       }
       __syncthreads();
       // suffix scan: thread t covers bins nb-1-kPerT*t-i, i < kPerT
@@ -449,6 +448,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_scatter_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const uint32_t* __restrict__ hist, int topk, uint64_t* __restrict__ cand,
     uint32_t* __restrict__ gcount) {
+  pdl_prologue();
   __shared__ uint8_t gid[kScoreHistBins];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t lcount[kMaxGroups], lbase[kMaxGroups];
@@ -498,6 +498,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const uint32_t* __restrict__ hist, int topk, const uint64_t* __restrict__ cand,
     int32_t* __restrict__ idx, float* __restrict__ vals) {
+  pdl_prologue();
   extern __shared__ uint64_t gbuf[];   // [2 * kGroupBuf]: gathered, then sorted
   __shared__ uint32_t buckets[kSubBucketWords];
   __shared__ uint32_t warp_sums[32];
@@ -601,6 +602,7 @@ __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const uint32_t* __restrict__ hist, int topk, int sortn, int32_t* __restrict__ idx,
     float* __restrict__ vals) {
+  pdl_prologue();
   extern __shared__ uint64_t sel[];   // [sortn]
   __shared__ uint32_t hbuf[kBins];
   __shared__ uint32_t warp_sums[32];
@@ -688,6 +690,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     const int32_t* __restrict__ gather_len, const int32_t* __restrict__ index_map,
     const uint32_t* __restrict__ ghist, int topk, int32_t* __restrict__ idx,
     float* __restrict__ vals, int* status, int64_t row0) {
+  pdl_prologue();
   using RC = RowCfg<NT, CAP, ROWCAP>;
   extern __shared__ __align__(128) uint64_t rbuf[];
   uint64_t* sorted = rbuf;                                     // [CAP] sorted pairs (later)
@@ -986,9 +989,9 @@ cudaError_t launch_row(const float* scores, int64_t stride, const int32_t* pos, 
   if (e != cudaSuccess) return e;
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
-    topk_row_kernel<NT, CAP, ROWCAP, MINB><<<(unsigned)nr, NT, RC::kSmem, st>>>(
-        scores, stride, pos, L, gather_len, index_map, ghist, topk, idx, vals, status, row0);
-    e = cudaGetLastError();
+    e = launch_pdl(topk_row_kernel<NT, CAP, ROWCAP, MINB>, dim3((unsigned)nr), dim3(NT),
+                   RC::kSmem, st, scores, stride, pos, L, gather_len, index_map, ghist, topk, idx,
+                   vals, status, row0);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -1009,26 +1012,23 @@ cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t*
     return launch_row<1024, 3072, kLongRowCap, 1>(scores, stride, pos, L, nullptr, nullptr, hist,
                                                   rows, topk, idx, vals, status, st);
   dim3 sgrid((unsigned)((L + kScatterChunk - 1) / kScatterChunk), (unsigned)rows);
-  topk_scatter_kernel<<<sgrid, kSelThreads, 0, st>>>(scores, stride, pos, L, hist, topk, cand,
-                                                     gcount);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(topk_scatter_kernel, sgrid, dim3(kSelThreads), 0, st, scores, stride,
+                             pos, L, hist, topk, cand, gcount);
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)2 * kGroupBuf * sizeof(uint64_t);
   e = cudaFuncSetAttribute(topk_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  topk_group_kernel<<<dim3(kMaxGroups, (unsigned)rows), kSelThreads, smem, st>>>(
-      scores, stride, pos, L, hist, topk, cand, idx, vals);
-  e = cudaGetLastError();
+  e = launch_pdl(topk_group_kernel, dim3(kMaxGroups, (unsigned)rows), dim3(kSelThreads), smem, st,
+                 scores, stride, pos, L, hist, topk, (const uint64_t*)cand, idx, vals);
   if (e != cudaSuccess || topk <= kGroupBuf) return e;   // the group kernel covers overflow rows
   const int sortn = topk_sort_size(topk);
   const size_t ov_smem = (size_t)sortn * sizeof(uint64_t);
   e = cudaFuncSetAttribute(topk_hist_overflow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)ov_smem);
   if (e != cudaSuccess) return e;
-  topk_hist_overflow_kernel<<<rows, kThreads, ov_smem, st>>>(scores, stride, pos, L, hist, topk,
-                                                             sortn, idx, vals);
-  return cudaGetLastError();
+  return launch_pdl(topk_hist_overflow_kernel, dim3(rows), dim3(kThreads), ov_smem, st, scores,
+                    stride, pos, L, hist, topk, sortn, idx, vals);
 }
 
 size_t topk_hist_ws_bytes(int64_t rows) {

@@ -57,6 +57,18 @@ def _dist_env():
     return rank, world, local
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's elapsed time (every rank passes its own; a collective that all ranks
+    take in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -338,11 +350,7 @@ def run_cuda(args, wl):
             step_fn(warmup + i, **kw)
         e1.record(stream)
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         return ms / steps
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)

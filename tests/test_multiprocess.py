@@ -1,0 +1,70 @@
+"""The multi-GPU path is replicas only (independent sequences, no exchange step): what there is
+to cover is the host logic around it, run here as world-size-2 process groups on the CPU with
+gloo.  Every rank times its own replica and the reported time is the slowest rank's; under
+torchrun the reference arm runs on rank 0 alone and the other ranks exit 0 without work."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_max(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    sys.path.insert(0, ROOT)
+    import bench
+    got = bench.max_over_ranks(10.0 + 5.0 * rank, world, "cpu")
+    dist.barrier()
+    dist.destroy_process_group()
+    out.put((rank, got))
+
+
+def test_max_over_ranks_takes_the_slowest_rank():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_max, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=5) for _ in range(world))
+    assert got == {0: 15.0, 1: 15.0}
+
+
+def test_single_rank_time_is_its_own():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
+
+
+@pytest.mark.slow
+def test_reference_arm_under_torchrun_prints_once():
+    """Two ranks launched the way the driver launches them: one JSON line, every rank exits 0."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--workload", "tiny_2k", "--steps", "1",
+           "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0

@@ -2,20 +2,26 @@
 // paper summary.  Output order: descending score, equal scores by ascending token
 // index; rows shorter than k are padded with index -1 and value -inf.
 //
-// Scores are mapped to order-preserving uint32 keys and the k-th largest key is found
-// exactly by a three-pass radix select (11, 11 and 10 bits; histograms in shared
-// memory, a block-wide suffix scan picks the bin).  A final pass in index order takes
-// every key above that threshold plus the lowest-index keys equal to it, so exactly k
-// (key, index) pairs remain; a bitonic sort of those 64-bit pairs in shared memory
-// gives the output order.
+// Scores are mapped to order-preserving uint32 keys (composite 64-bit pairs with the
+// complemented index, so equal keys order by ascending index).  The forms, by row shape:
 //
-// topk_cluster_kernel (main form): a row is split over a thread-block cluster of G CTAs
-// (G = 1, 2, 4 or 8).  Each CTA reads its slice of the row from global memory once and
-// keeps it in shared memory as keys; the per-pass histograms are summed across the
-// cluster through distributed shared memory, so every CTA picks the same digit, and
-// the selected pairs are written straight into the leader CTA's sort buffer.
+// topk_row_kernel (rows up to 16384 scores, or 40960 with the scorer's histogram): one CTA
+// per row stages the row in shared memory with one bulk copy, finds the cutoff bin of a
+// 12-bit key histogram (refined by the next 12 bits when the bin is crowded), compacts the
+// candidates and sorts them with a histogram-adaptive counting sort (groupsort.cuh).
+//
+// topk_scatter_kernel + topk_group_kernel (longer decode rows with the scorer's histogram):
+// many CTAs per row append the candidates to groups of output positions, one CTA per group
+// sorts them; topk_hist_overflow_kernel takes rows whose candidates do not fit the groups.
+//
+// topk_cluster_kernel (other long rows): a row is split over a thread-block cluster of G
+// CTAs (G = 1, 2, 4 or 8).  Each CTA keeps its slice of the row in shared memory as keys;
+// the k-th largest key is found exactly by a three-pass radix select (11, 11 and 10 bits)
+// whose per-pass histograms are summed across the cluster through distributed shared
+// memory; the selected pairs (every key above the threshold plus the lowest-index keys
+// equal to it) go to the leader CTA, which sorts them.
 // topk_kernel (fallback for rows too long for a cluster's shared memory): one CTA per
-// row, every pass re-reads the row from global memory.
+// row, every radix pass re-reads the row from global memory.
 #include <cooperative_groups.h>
 
 #include "blocksort.cuh"

@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -79,11 +80,16 @@ class ClockSampler:
     def __init__(self, gpu_id: str, tag: int):
         self.gpu = gpu_id            # nvidia-smi --id value (the device UUID)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{tag}.csv")
+        out_dir = os.environ.get("MISA_BENCH_LOG_DIR")   # keep the raw samples there if set
+        if out_dir:
+            self.path = os.path.join(out_dir, f"clocks_rank{tag}.csv")
+        else:
+            fd, self.path = tempfile.mkstemp(prefix=f"misa_clocks_rank{tag}_", suffix=".csv")
+            os.close(fd)
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(self.path) or ".", exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",

@@ -56,7 +56,7 @@ def test_single_rank_time_is_its_own():
 
 @pytest.mark.slow
 def test_reference_arm_under_torchrun_prints_once():
-    """Two ranks launched the way the driver launches them: one JSON line, every rank exits 0."""
+    """Two ranks under torchrun on one node: one JSON line, every rank exits 0."""
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",

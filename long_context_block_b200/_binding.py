@@ -106,7 +106,11 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
 
 
 class _Workspace:
-    """One zero-initialised scratch buffer per device, grown on demand."""
+    """One zero-initialised scratch buffer per device, grown on demand.
+
+    Every call on a device uses this buffer, so (as the C ABI requires of one workspace)
+    calls issued on different streams must not overlap on the GPU: synchronise the streams
+    between them, or call the C entry points with a workspace per stream."""
 
     def __init__(self):
         self._buf = {}

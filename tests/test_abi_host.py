@@ -59,6 +59,28 @@ def test_workspace_sizes(lib):
     assert ws(9, 1, 1, 64, 128, 1024, 64, 8, 16, 16) == 0
 
 
+def test_workspace_sizes_of_query_blocks(lib):
+    """A sequence with T >= 2 queries is scored in units of QB queries (QB = the next power of
+    two >= T, at most 256 / HS, at least 32 columns), HS = routed heads rounded up to a power
+    of two >= 8: the scorer scratch holds units x QB x HS gathered rows."""
+    ws = lib.misa_workspace_size
+    a256 = lambda x: (x + 255) // 256 * 256
+    tc = lambda units, n: a256(units * n * 256) + a256(units * n * 4) + a256((units + 1) * 4)
+    L = 4096   # below the histogram path's 8192, so no histogram scratch
+    for T, h, units, n in ((2, 8, 1, 32),     # QB = 4 (32 columns at HS = 8)
+                           (3, 8, 1, 32),
+                           (5, 8, 1, 64),     # QB = 8
+                           (16, 8, 1, 128),
+                           (40, 8, 2, 256),   # full width: QB = 32
+                           (2, 16, 1, 32),    # HS = 16, QB = 2
+                           (9, 16, 1, 256)):  # QB = 16
+        assert ws(2, 1, T, 64, 128, L, 64, h, 256, 512) == 256 + T * L * 4 + tc(units, n), (T, h)
+    # several sequences: units per sequence times nseq
+    assert ws(2, 3, 4, 64, 128, L, 64, 8, 256, 512) == 256 + 12 * L * 4 + tc(3, 32)
+    # dense DSA (all 64 heads, HS = 64): 4 queries fill a 256-column unit
+    assert ws(3, 1, 4, 64, 128, L, 64, 8, 256, 512) == 256 + 4 * L * 4 + tc(1, 256)
+
+
 def test_invalid_arguments_rejected_on_host(lib):
     c = lib.library()
     null = None

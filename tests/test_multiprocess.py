@@ -68,3 +68,18 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_reference_arm_line_contract():
+    """The reference arm on one process: the oracle timed on the host, with its cpu_baseline
+    and an e2e object that moves no bytes to or from a device."""
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny_2k",
+           "--steps", "2", "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 1 and line["steps"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["unit"] == line["unit"]
+    assert line["higher_is_better"] is True and line["config"]["workload"] == "tiny_2k"

@@ -32,7 +32,10 @@ design notes of the repository):
     index first.  When fewer than k items exist, all are returned and the rest of
     the row is padded with -1 (values -inf).
   * MISA-dagger's fine stage recomputes the full all-head score I[t,s] for every
-    candidate; ties there are broken by the lower token index s.
+    candidate; ties there are broken by the lower token index s.  Omega_t is a set
+    (Eq. 11 selects it by TopK, Eq. 12 ranges over s in Omega_t): a candidate list
+    handed in with a repeated id counts that id once, and -1 marks an empty slot;
+    ids outside the query's prefix [0, P) are not tokens of Omega_t and are dropped.
   * Precision: q and k are bf16 values, w is fp32; everything here is widened to
     float64 and computed in float64.
 
@@ -48,7 +51,6 @@ import numpy as np
 __all__ = [
     "bf16_bits_to_f64", "pool_keys", "router_energy", "select_heads", "token_scores",
     "dense_scores", "topk", "misa_row", "dsa_row", "misa_dagger_row", "recall",
-    "oracle_rows",
 ]
 
 
@@ -150,12 +152,17 @@ def dsa_row(q_t, w_t, k, P, kk):
 
 
 def misa_dagger_row(q_t, w_t, k, P, cand, kk):
-    """MISA-dagger fine stage (Eq. 12) for candidate tokens `cand` (-1 entries ignored)."""
+    """MISA-dagger fine stage (Eq. 12) over the candidate set Omega_t given by `cand`.
+
+    `cand` may list an id more than once and in any order; -1 marks an empty slot.
+    Omega_t is the set of distinct ids in [0, P).  Returns idx / vals of the TopK, and
+    the set itself ("cand", ascending) with the all-head scores of its members ("scores").
+    """
     c = np.asarray(cand, dtype=np.int64)
-    c = c[c >= 0]
+    c = np.unique(c[(c >= 0) & (c < P)])                # Omega_t as a set, ascending
     s_full = dense_scores(q_t, w_t, k[c], c.shape[0])   # I[t, s] for s in Omega_t
     idx, vals = topk(s_full, kk, index=c)
-    return dict(idx=idx, vals=vals)
+    return dict(idx=idx, vals=vals, cand=c, scores=s_full)
 
 
 def recall(sel: np.ndarray, ref: np.ndarray) -> float:
@@ -163,44 +170,3 @@ def recall(sel: np.ndarray, ref: np.ndarray) -> float:
     a = set(int(x) for x in sel if x >= 0)
     b = set(int(x) for x in ref if x >= 0)
     return len(a & b) / max(1, len(b))
-
-
-# --------------------------------------------------------------------------- batch helper
-def oracle_rows(q_bits, w, k_bits, pos, rows, B, h, kk, kprime=None, heads_given=None,
-                with_dense=True):
-    """Run the oracle on flat query rows (row = seq * T + t) of a batch.
-
-    Returns a list of dicts with the per-row results of MISA (routed with the
-    oracle's own heads), optionally the routed scores under `heads_given[row]`,
-    dense DSA, and MISA-dagger (coarse stage = the oracle's own MISA scores).
-    """
-    nseq, T, H, d = q_bits.shape
-    out = []
-    kcache = {}
-    for row in rows:
-        n, t = divmod(int(row), T)
-        if n not in kcache:
-            kcache.clear()
-            kcache[n] = bf16_bits_to_f64(k_bits[n])
-        k = kcache[n]
-        q_t = bf16_bits_to_f64(q_bits[n, t])
-        w_t = np.asarray(w[n, t], dtype=np.float64)
-        P = int(pos[n, t]) + 1
-        r = misa_row(q_t, w_t, k, P, B, h, kk)
-        r["row"] = int(row)
-        r["P"] = P
-        if heads_given is not None:
-            r["scores_given_heads"] = token_scores(q_t, w_t, k, P, heads_given[int(row)])
-        if with_dense:
-            dd = dsa_row(q_t, w_t, k, P, kk)
-            r["dense_scores"] = dd["scores"]
-            r["dense_idx"] = dd["idx"]
-            r["dense_vals"] = dd["vals"]
-        if kprime is not None:
-            cidx, _ = topk(r["scores"], kprime)
-            r["cand"] = cidx
-            dg = misa_dagger_row(q_t, w_t, k, P, cidx, kk)
-            r["dagger_idx"] = dg["idx"]
-            r["dagger_vals"] = dg["vals"]
-        out.append(r)
-    return out

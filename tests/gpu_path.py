@@ -102,9 +102,10 @@ def check_rows(x, host, rows, B, h, topk, kprime, check_pool=True):
         tl.check_scores(host["dvals"][i][:dsel.size], d_ref[dsel], what=f"{tag} DSA vals")
         # MISA-dagger: coarse candidates (Eq. 11) then all-head re-rank (Eq. 12)
         tl.check_selection(host["cand"][i], s_ref, kprime, what=f"{tag} MISA-dagger candidates")
-        c = host["cand"][i][host["cand"][i] >= 0]
-        stats["dagger_swaps"] += tl.check_selection(host["gidx"][i], d_ref[c], topk,
-                                                    what=f"{tag} MISA-dagger top-k", ids=c)
+        dg = orc.misa_dagger_row(q_t, w_t, k, P, host["cand"][i], topk)
+        stats["dagger_swaps"] += tl.check_selection(host["gidx"][i], dg["scores"], topk,
+                                                    what=f"{tag} MISA-dagger top-k",
+                                                    ids=dg["cand"])
         tl.check_order(host["gidx"][i], host["gvals"][i], what=f"{tag} MISA-dagger order")
         gsel = host["gidx"][i][host["gidx"][i] >= 0]
         tl.check_scores(host["gvals"][i][:gsel.size], d_ref[gsel], what=f"{tag} MISA-dagger vals")

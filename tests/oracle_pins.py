@@ -5,6 +5,8 @@ run against deliberately broken copies of the oracle (see test_oracle_mutations.
 to show that a plausible mistake is caught.
 
 Sources of truth used here:
+  * the bf16 format itself: torch's own bf16 -> float64 conversion over all 65,536 bit
+    patterns, and values fixed by the format (1.0, -2.0, the smallest subnormal, inf);
   * hand-worked examples of Eqs. (1), (2), (4), (7)-(12) in tests/golden/
     ("MISA: Mixture of Indexer Sparse Attention", Introduction and Methodology);
   * closed forms (the mean of an arithmetic progression of keys);
@@ -199,7 +201,61 @@ def check_causal_prefix(orc):
     assert r1["scores"].shape == (50,)
 
 
+# ----------------------------------------------------------------- input widening and reporting
+def check_bf16_widening(orc):
+    """bf16 bit patterns widen to the float64 value the bf16 format defines: compared with
+    torch's bf16 -> float64 conversion on every non-NaN pattern, and with values the format
+    fixes by hand (sign, exponent bias 127, 7 stored mantissa bits, subnormals)."""
+    import torch
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    with np.errstate(invalid="ignore"):   # the NaN patterns
+        got = orc.bf16_bits_to_f64(bits)
+    assert got.dtype == np.float64 and got.shape == (1 << 16,)
+    keep = ~np.isnan(ref)
+    assert np.array_equal(got[keep], ref[keep]), np.nonzero(got[keep] != ref[keep])[0][:5]
+    assert np.all(np.isnan(got[~keep]))
+    hand = {0x3F80: 1.0, 0xC000: -2.0, 0x3FC0: 1.5, 0x0001: 2.0 ** -133, 0x8000: -0.0,
+            0x7F80: np.inf, 0xFF80: -np.inf, 0x4049: 3.140625, 0x0080: 2.0 ** -126}
+    for b, v in hand.items():
+        w = orc.bf16_bits_to_f64(np.array([b], dtype=np.uint16))[0]
+        assert w == v and np.signbit(w) == np.signbit(v), (hex(b), w, v)
+    # shape is kept for multi-dimensional inputs
+    assert orc.bf16_bits_to_f64(np.full((2, 3), 0x3F80, dtype=np.uint16)).shape == (2, 3)
+
+
+def check_recall_hand(orc):
+    """recall = |sel intersect ref| / |ref| over valid (>= 0) ids: the fraction of the
+    dense selection that the other selection recovers (the pages' token-recovery measure)."""
+    assert orc.recall(np.array([5, 2, 9, 11]), np.array([2, 9, 7])) == 2 / 3
+    # padding (-1) is not a token on either side
+    assert orc.recall(np.array([-1, 4, -1]), np.array([4, 8, -1, -1])) == 1 / 2
+    assert orc.recall(np.array([1, 2, 3]), np.array([3, 2, 1])) == 1.0
+    assert orc.recall(np.array([-1, -1]), np.array([6, 7])) == 0.0
+
+
+def check_dagger_candidate_set(orc):
+    """Eq. (12) ranges over the set Omega_t: a repeated candidate id counts once and -1
+    slots are empty.  Hand case: H = 1, d = 1, w = 1, q = 1, keys k_s = s, so I[s] = s.
+    Candidates [3, 3, 1, -1, 3, 0] form {0, 1, 3}; TopK(., 2) = [3, 1].  Counting the
+    repeats would return [3, 3]."""
+    q = np.array([[1.0]])
+    w = np.array([1.0])
+    k = np.arange(6, dtype=np.float64)[:, None]
+    dg = orc.misa_dagger_row(q, w, k, 6, np.array([3, 3, 1, -1, 3, 0]), 2)
+    assert list(dg["idx"]) == [3, 1], dg["idx"]
+    assert list(dg["vals"]) == [3.0, 1.0]
+    assert list(dg["cand"]) == [0, 1, 3] and list(dg["scores"]) == [0.0, 1.0, 3.0]
+    # fewer distinct candidates than k: padded with -1 / -inf
+    dg = orc.misa_dagger_row(q, w, k, 6, np.array([2, 2, 2, -1]), 3)
+    assert list(dg["idx"]) == [2, -1, -1] and np.all(np.isneginf(dg["vals"][1:]))
+    # ids past the query's prefix (P = 4) are not tokens of Omega_t
+    dg = orc.misa_dagger_row(q, w, k, 4, np.array([5, 1, 4, 2]), 2)
+    assert list(dg["idx"]) == [2, 1], dg["idx"]
+
+
 ALL_CHECKS = [
+    check_bf16_widening, check_recall_hand, check_dagger_candidate_set,
     check_dense_hand, check_router_hand, check_pool_closed_form, check_router_closed_form,
     check_partial_block_router, check_topk_against_library, check_topk_brute_rank,
     check_h_equals_H_is_dense, check_dagger_limits, check_router_w_invariance,

@@ -213,10 +213,12 @@ def test_dagger_candidates_any_order_with_repeats(M):
         for t in range(wl.T):
             P = int(x.pos[n, t]) + 1
             q_t = orc.bf16_bits_to_f64(x.q_bits[n, t])
-            d_ref = orc.dense_scores(q_t, x.w[n, t].astype(np.float64), kk, P)
-            c = np.unique(cand[n, t][cand[n, t] >= 0])
+            w_t = x.w[n, t].astype(np.float64)
+            d_ref = orc.dense_scores(q_t, w_t, kk, P)
+            dg = orc.misa_dagger_row(q_t, w_t, kk, P, cand[n, t], wl.topk)   # Omega_t as a set
             assert len(set(idx[n, t].tolist())) == wl.topk
-            tl.check_selection(idx[n, t], d_ref[c], wl.topk, what=f"dagger {n},{t}", ids=c)
+            tl.check_selection(idx[n, t], dg["scores"], wl.topk, what=f"dagger {n},{t}",
+                               ids=dg["cand"])
             tl.check_order(idx[n, t], vals[n, t], what=f"dagger order {n},{t}")
             tl.check_scores(vals[n, t], d_ref[idx[n, t]], what=f"dagger vals {n},{t}")
 

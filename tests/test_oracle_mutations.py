@@ -64,7 +64,55 @@ def _heads_ascending(E, h):
     return np.argsort(E, kind="stable")[:h]
 
 
+def _bf16_shift15(bits):
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)
+
+
+def _bf16_as_fp16(bits):
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def _bf16_truncated_mantissa(bits):
+    b = np.asarray(bits, dtype=np.uint16) & np.uint16(0xFFF0)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def _recall_over_sel(sel, ref):
+    a = set(int(x) for x in sel if x >= 0)
+    b = set(int(x) for x in ref if x >= 0)
+    return len(a & b) / max(1, len(a))
+
+
+def _recall_counts_padding(sel, ref):
+    a, b = set(int(x) for x in sel), set(int(x) for x in ref)
+    return len(a & b) / max(1, len(b))
+
+
+def _dagger_keeps_repeats(q_t, w_t, k, P, cand, kk):
+    c = np.asarray(cand, dtype=np.int64)
+    c = c[c >= 0]
+    s_full = orc.dense_scores(q_t, w_t, k[c], c.shape[0])
+    idx, vals = orc.topk(s_full, kk, index=c)
+    return dict(idx=idx, vals=vals, cand=c, scores=s_full)
+
+
+def _dagger_ignores_prefix(q_t, w_t, k, P, cand, kk):
+    c = np.asarray(cand, dtype=np.int64)
+    c = np.unique(c[c >= 0])
+    s_full = orc.dense_scores(q_t, w_t, k[c], c.shape[0])
+    idx, vals = orc.topk(s_full, kk, index=c)
+    return dict(idx=idx, vals=vals, cand=c, scores=s_full)
+
+
 MUTANTS = [
+    ("bf16_bits_to_f64", _bf16_shift15),
+    ("bf16_bits_to_f64", _bf16_as_fp16),
+    ("bf16_bits_to_f64", _bf16_truncated_mantissa),
+    ("recall", _recall_over_sel),
+    ("recall", _recall_counts_padding),
+    ("misa_dagger_row", _dagger_keeps_repeats),
+    ("misa_dagger_row", _dagger_ignores_prefix),
     ("token_scores", _relu_after_weight),
     ("token_scores", _no_relu),
     ("token_scores", _transposed_q),
@@ -84,6 +132,6 @@ def test_pins_catch_planted_mistake(monkeypatch, name, fn):
     for check in oracle_pins.ALL_CHECKS:
         try:
             check(orc)
-        except (AssertionError, ValueError, IndexError):
+        except (AssertionError, ValueError, IndexError, TypeError, KeyError):
             caught.append(check.__name__)
     assert caught, f"no pin caught the planted mistake {fn.__name__}"

@@ -20,6 +20,11 @@ Long-Context LLM Inference" (picx.dev summary page):
   * Eq. (10) final selection TopK_s(Ihat[t,:], k)
   * Eq. (11) MISA-dagger coarse candidates Omega_t = TopK_s(Ihat[t,:], k')
   * Eq. (12) MISA-dagger fine stage TopK over s in Omega_t of I[t,s]
+  * the HISA-style token-axis filter the page contrasts MISA with ("Key distinction
+    from HISA", Methodology section 1): the same affinities A[t,j,b], reduced across
+    heads instead of across blocks, pick the top-m blocks; the original indexer then
+    scores only the tokens of those blocks (the two-stage search the HISA abstract
+    describes: block-level coarse filter, token-level refinement in the kept blocks).
 
 Readings taken where the page is silent (each listed with its reason in the
 design notes of the repository):
@@ -51,6 +56,7 @@ import numpy as np
 __all__ = [
     "bf16_bits_to_f64", "pool_keys", "router_energy", "select_heads", "token_scores",
     "dense_scores", "topk", "misa_row", "dsa_row", "misa_dagger_row", "recall",
+    "block_scores", "hisa_row",
 ]
 
 
@@ -163,6 +169,34 @@ def misa_dagger_row(q_t, w_t, k, P, cand, kk):
     s_full = dense_scores(q_t, w_t, k[c], c.shape[0])   # I[t, s] for s in Omega_t
     idx, vals = topk(s_full, kk, index=c)
     return dict(idx=idx, vals=vals, cand=c, scores=s_full)
+
+
+# --------------------------------------------------------------------------- HISA-style filter
+def block_scores(q_t: np.ndarray, w_t: np.ndarray, k: np.ndarray, P: int, B: int) -> np.ndarray:
+    """Head-axis reduction of the router affinities: G[b] = sum_j A[j, b] with
+    A[j, b] = w_j * ReLU(q_j . kpool_b) over the blocks of the query's prefix (the same
+    blocks, partial last block included, as Eq. 7).  Returns float64 [ceil(P/B)]."""
+    kpool = pool_keys(k[:P], B)                         # [M, d]
+    A = w_t[:, None] * np.maximum(q_t @ kpool.T, 0.0)   # [H, M]
+    G = np.zeros(kpool.shape[0], dtype=np.float64)
+    for j in range(A.shape[0]):                         # sum over heads in ascending j
+        G += A[j]
+    return G
+
+
+def hisa_row(q_t, w_t, k, P, B, m, kk):
+    """Token-axis block filter for one query: keep the m blocks with the largest G[b]
+    (ties: lower b), then TopK of the all-head score I[t,s] (Eq. 1) over the tokens of
+    the kept blocks (ties: lower s).  Returns the block scores, the kept blocks (by
+    descending G), the candidate tokens (ascending) with their scores, and idx / vals."""
+    G = block_scores(q_t, w_t, k, P, B)
+    blocks, _ = topk(G, m)
+    blocks = blocks[blocks >= 0]
+    toks = [np.arange(b * B, min((b + 1) * B, P)) for b in sorted(int(b) for b in blocks)]
+    cand = np.concatenate(toks).astype(np.int64) if toks else np.zeros(0, dtype=np.int64)
+    s = dense_scores(q_t, w_t, k[cand], cand.shape[0])
+    idx, vals = topk(s, kk, index=cand)
+    return dict(G=G, blocks=blocks, cand=cand, scores=s, idx=idx, vals=vals)
 
 
 def recall(sel: np.ndarray, ref: np.ndarray) -> float:

@@ -254,7 +254,47 @@ def check_dagger_candidate_set(orc):
     assert list(dg["idx"]) == [2, 1], dg["idx"]
 
 
+# ----------------------------------------------------------------- HISA-style block filter
+def check_hisa_hand(orc):
+    """Hand case of the head-axis reduction G[b] = sum_j A[j, b] (MISA page, "Key
+    distinction from HISA"): H = 2, d = 2, B = 2, P = 7, q = I, w = (1, -0.5),
+    keys (1,0) (3,0) (0,2) (0,4) (2,2) (0,0) (5,-1).  Pooled keys of the prefix:
+    (2,0) (0,3) (1,1) and the partial block {6}: (5,-1).  A[0,:] = (2, 0, 1, 5),
+    A[1,:] = (0, -1.5, -0.5, 0), so G = (2, -1.5, 0.5, 5).  Top-3 blocks: 3, 0, 2; their
+    tokens 0 1 4 5 6 have dense scores 1 3 1 0 5, so TopK(., 2) = [6, 1]."""
+    q = np.eye(2)
+    w = np.array([1.0, -0.5])
+    k = np.array([[1, 0], [3, 0], [0, 2], [0, 4], [2, 2], [0, 0], [5, -1], [9, 9]], float)
+    assert np.array_equal(orc.block_scores(q, w, k, 7, 2), [2.0, -1.5, 0.5, 5.0])
+    r = orc.hisa_row(q, w, k, 7, 2, 3, 2)
+    assert list(r["blocks"]) == [3, 0, 2], r["blocks"]
+    assert list(r["cand"]) == [0, 1, 4, 5, 6], r["cand"]
+    assert list(r["scores"]) == [1.0, 3.0, 1.0, 0.0, 5.0], r["scores"]
+    assert list(r["idx"]) == [6, 1] and list(r["vals"]) == [5.0, 3.0]
+    # two blocks: 3 and 0 -> tokens 0 1 6; TopK(., 3) = [6, 1, 0]
+    r = orc.hisa_row(q, w, k, 7, 2, 2, 3)
+    assert list(r["blocks"]) == [3, 0] and list(r["idx"]) == [6, 1, 0], r["idx"]
+    # more blocks than the prefix has: every token, padded past P
+    r = orc.hisa_row(q, w, k, 3, 2, 5, 4)
+    assert list(r["cand"]) == [0, 1, 2] and list(r["idx"]) == [1, 0, 2, -1], r["idx"]
+
+
+def check_hisa_limits(orc):
+    """m >= M keeps every block, so the filter is the dense TopK exactly; with B = 1 every
+    block is one token and G is the dense score itself, so m = k returns DSA's selection."""
+    for seed in range(4):
+        q, w, k = _rand_problem(seed + 40)
+        for P in (1, 30, 97):
+            M = -(-P // 8)
+            r = orc.hisa_row(q, w, k, P, 8, M, 10)
+            assert np.array_equal(r["idx"], orc.dsa_row(q, w, k, P, 10)["idx"])
+            assert np.array_equal(orc.block_scores(q, w, k, P, 1), orc.dense_scores(q, w, k, P))
+            r1 = orc.hisa_row(q, w, k, P, 1, 10, 10)
+            assert np.array_equal(r1["idx"], orc.dsa_row(q, w, k, P, 10)["idx"])
+
+
 ALL_CHECKS = [
+    check_hisa_hand, check_hisa_limits,
     check_bf16_widening, check_recall_hand, check_dagger_candidate_set,
     check_dense_hand, check_router_hand, check_pool_closed_form, check_router_closed_form,
     check_partial_block_router, check_topk_against_library, check_topk_brute_rank,

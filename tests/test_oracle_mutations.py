@@ -105,7 +105,37 @@ def _dagger_ignores_prefix(q_t, w_t, k, P, cand, kk):
     return dict(idx=idx, vals=vals, cand=c, scores=s_full)
 
 
+def _block_scores_abs(q_t, w_t, k, P, B):
+    kp = orc.pool_keys(k[:P], B)
+    return np.abs(w_t[:, None] * np.maximum(q_t @ kp.T, 0.0)).sum(axis=0)
+
+
+def _block_scores_drop_partial(q_t, w_t, k, P, B):
+    Pf = max(B, (P // B) * B) if P >= B else P
+    kp = orc.pool_keys(k[:Pf], B)
+    return (w_t[:, None] * np.maximum(q_t @ kp.T, 0.0)).sum(axis=0)
+
+
+def _block_scores_relu_after_sum(q_t, w_t, k, P, B):
+    kp = orc.pool_keys(k[:P], B)
+    return np.maximum((w_t[:, None] * (q_t @ kp.T)).sum(axis=0), 0.0)
+
+
+def _hisa_lowest_blocks(q_t, w_t, k, P, B, m, kk):
+    G = orc.block_scores(q_t, w_t, k, P, B)
+    blocks = np.argsort(G, kind="stable")[:m]
+    toks = [np.arange(b * B, min((b + 1) * B, P)) for b in sorted(int(b) for b in blocks)]
+    cand = np.concatenate(toks).astype(np.int64)
+    s = orc.dense_scores(q_t, w_t, k[cand], cand.shape[0])
+    idx, vals = orc.topk(s, kk, index=cand)
+    return dict(G=G, blocks=blocks, cand=cand, scores=s, idx=idx, vals=vals)
+
+
 MUTANTS = [
+    ("block_scores", _block_scores_abs),
+    ("block_scores", _block_scores_drop_partial),
+    ("block_scores", _block_scores_relu_after_sum),
+    ("hisa_row", _hisa_lowest_blocks),
     ("bf16_bits_to_f64", _bf16_shift15),
     ("bf16_bits_to_f64", _bf16_as_fp16),
     ("bf16_bits_to_f64", _bf16_truncated_mantissa),

@@ -211,7 +211,8 @@ def run_reference(args, wl):
         "data": "synthetic",
         "config": {"workload": wl.name, "nseq": wl.nseq, "T": wl.T, "L": wl.L, "H": wl.H,
                    "h": wl.h, "B": wl.B, "topk": wl.topk, "path": "MISA (pool+route+score+top-k)"},
-        "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads,
+                         "host_cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"{args.steps} query rows of {wl.name} (one row per step), "
                                    "fp64 numpy oracle"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -241,22 +242,42 @@ def cpu_baseline(wl, budget_s: float = 10.0):
             break
     dt = time.perf_counter() - t0
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    return {"value": units / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+    return {"value": units / dt, "unit": UNIT, "cores": threads,
+            "host_cores": os.cpu_count(), "kind": "oracle",
             "sample": f"{rows_done} query rows of {wl.name} ({units} query x prefix-token pairs), "
                       f"full MISA path in fp64 numpy, {dt:.1f} s"}
 
 
-def run_cuda(args, wl):
+EXTRA_WORKLOADS = ("dsv32_prefill_16k", "glm5_decode_128k", "dagger_128k")
+
+
+def _roofline(wl, ms_score_kernel, peaks, traffic):
+    """Roofline object of the routed scorer: its bound is whichever of the kernel's
+    algorithmic flops and bytes takes longer at the measured peaks."""
+    flops = algorithmic_flops_score(wl)
+    score_bytes = algorithmic_bytes_score(wl)
+    form = "block form" if block_form(wl) else "decode form"
+    common = {"kernel": f"score_tc_kernel (routed scoring, {form})", "traffic": traffic,
+              "algorithmic_flops": flops, "algorithmic_bytes": score_bytes,
+              "avg_ms": ms_score_kernel}
+    if flops / (peaks["bf16"] * 1e12) > score_bytes / (peaks["hbm"] * 1e9):
+        achieved = flops / (ms_score_kernel * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16"],
+                "peak_source": peaks["source"] + " bf16 dense (burst)", **common}
+    achieved = score_bytes / (ms_score_kernel * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm"], "peak_source": peaks["source"] + " HBM copy",
+            **common}
+
+
+def measure_workload(M, wl, args, dev, world, rank, peaks, headline: bool):
+    """Time MISA, dense DSA, MISA-dagger (and, for decode, MISA with kept pooled keys) on
+    one workload with two resident input copies used alternately; also the routed scorer
+    alone (for the roofline), recall against DSA and the clocks during the MISA region.
+    The headline workload also gets the end-to-end number.  Returns (result, misa_ms)."""
     import torch
     import torch.distributed as dist
-    rank, world, local = _dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
-                                device_id=dev)
-    import long_context_block_b200 as M
-    peaks = _peaks()
 
     x = make_inputs(wl, seed=rank)
     q_h = torch.from_numpy(x.q_bits.view(np.int16)).pin_memory()
@@ -310,6 +331,23 @@ def run_cuda(args, wl):
         q, w, k, pos = sets[i % 2]
         M.dsa_score_topk(q, w, k, pos, wl.topk, idx=didx, vals=dvals)
 
+    # HISA-style block filter (decode workloads): the page's HISA block size B = 128 and
+    # m = k' / B blocks, so its token refinement re-scores as many tokens as MISA-dagger's
+    hisa_B = 128
+    hisa_m = max(1, wl.kprime // hisa_B)
+    hisa_on = T == 1
+    if hisa_on:
+        kp_h = [torch.empty((nseq, -(-wl.L // hisa_B), d), dtype=torch.float32, device=dev)
+                for _ in range(2)]
+        hidx = torch.empty_like(idx)
+        hvals = torch.empty_like(vals)
+
+    def hisa_step(i):
+        q, w, k, pos = sets[i % 2]
+        M.misa_pool_keys(k, hisa_B, out=kp_h[i % 2])
+        M.hisa_block_filter_topk(q, w, k, kp_h[i % 2], pos, hisa_B, hisa_m, wl.topk, idx=hidx,
+                                 vals=hvals)
+
     def kept_pool_step(i):
         # decode with the pooled keys kept between steps: each sequence's newest key (the
         # query's own position, L - 1) is the only change, so only its block is re-pooled
@@ -320,17 +358,13 @@ def run_cuda(args, wl):
 
     if args.only:
         # one path's steps and nothing else (for profiler captures); prints no bench line
-        fn = {"misa": misa_step, "dagger": dagger_step, "dsa": dsa_step}[args.only]
+        fn = {"misa": misa_step, "dagger": dagger_step, "dsa": dsa_step,
+              "kept": kept_pool_step, "hisa": hisa_step}[args.only]
         for i in range(args.warmup + args.steps):
             fn(i)
         torch.cuda.synchronize()
         M.misa_check_device_status(dev)
-        if world > 1:
-            dist.destroy_process_group()
-        if rank == 0:
-            print(json.dumps({"only": args.only, "workload": wl.name,
-                              "steps": args.warmup + args.steps}))
-        return 0
+        return {"only": args.only, "workload": wl.name, "steps": args.warmup + args.steps}, None
 
     def barrier():
         if world > 1:
@@ -345,7 +379,7 @@ def run_cuda(args, wl):
             t_end = time.perf_counter() + load_s
             i = warmup
             while time.perf_counter() < t_end:
-                for _ in range(50):
+                for _ in range(20):
                     step_fn(i)
                     i += 1
                 torch.cuda.synchronize()
@@ -360,35 +394,45 @@ def run_cuda(args, wl):
         return ms / steps
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    with ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid, rank) as clk:
-        ms_misa = timed(misa_step, args.steps, args.warmup, load_s=2.0, record=True)
+    with ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid,
+                      f"{rank}_{wl.name}") as clk:
+        ms_misa = timed(misa_step, args.steps, args.warmup, load_s=2.0 if headline else 1.0,
+                        record=True)
     clocks = clk.summary()
     M.misa_check_device_status(dev)
     per_call = [[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in ev_calls]
     call_ms = [sum(c[j] for c in per_call) / len(per_call) for j in range(3)]
-    score_ms_avg = call_ms[2]
     ms_dagger = timed(dagger_step, args.steps, args.warmup)
     ms_dsa = timed(dsa_step, args.steps, args.warmup)
     decode = T == 1 and bool(np.all(x.pos == wl.L - 1))
     ms_kept = timed(kept_pool_step, args.steps, args.warmup) if decode else None
+    ms_hisa = timed(hisa_step, args.steps, args.warmup) if hisa_on else None
 
     # selection agreement with dense DSA on the same inputs (outside the timed regions): the
     # fraction of DSA's k tokens that MISA and MISA-dagger also select, averaged over rows
     misa_step(0)
     dsa_step(0)
     dagger_step(0)
+    if hisa_on:
+        hisa_step(0)
     torch.cuda.synchronize()
 
     def recall(sel, ref):
         r = ref.reshape(-1, ref.shape[-1]).long()
         s_ = sel.reshape(-1, sel.shape[-1]).long()
-        mask = torch.zeros((r.shape[0], wl.L + 1), dtype=torch.bool, device=dev)
-        mask.scatter_(1, torch.where(r >= 0, r, wl.L), True)
-        hit = mask.gather(1, torch.where(s_ >= 0, s_, wl.L)) & (s_ >= 0)
-        n_ref = (r >= 0).sum(1).clamp(min=1)
-        return float((hit.sum(1).float() / n_ref.float()).mean().item())
+        out = []
+        for r0 in range(0, r.shape[0], 1024):   # bounded memory for many rows
+            rr, ss = r[r0:r0 + 1024], s_[r0:r0 + 1024]
+            mask = torch.zeros((rr.shape[0], wl.L + 1), dtype=torch.bool, device=dev)
+            mask.scatter_(1, torch.where(rr >= 0, rr, wl.L), True)
+            hit = mask.gather(1, torch.where(ss >= 0, ss, wl.L)) & (ss >= 0)
+            n_ref = (rr >= 0).sum(1).clamp(min=1)
+            out.append(hit.sum(1).float() / n_ref.float())
+        return float(torch.cat(out).mean().item())
 
     recalls = {"misa": recall(idx, didx), "misa_dagger": recall(gidx, didx)}
+    if hisa_on:
+        recalls["hisa_block_filter"] = recall(hidx, didx)
     # the routed scoring kernel alone (misa_score_rows: the scorer of misa_score_topk with the
     # same launch configuration), on the heads the MISA steps routed
     score_buf = torch.empty((nseq, T, wl.L), dtype=torch.float32, device=dev)
@@ -401,81 +445,110 @@ def run_cuda(args, wl):
     del score_buf
     M.misa_check_device_status(dev)
 
-    # end to end through the public API: pinned host inputs -> device -> MISA -> host indices
-    idx_h = torch.empty((nseq, T, wl.topk), dtype=torch.int32).pin_memory()
-    e2e_dev = [torch.empty_like(t) for t in sets[0]]
-
-    def e2e_step(i):
-        for dst, src in zip(e2e_dev, (q_h, w_h, k_h, pos_h)):
-            dst.view(src.dtype).copy_(src, non_blocking=True)
-        q, w, k, pos = e2e_dev
-        out_idx, _, _ = M.misa_indexer(q, w, k, pos, wl.B, wl.h, wl.topk)
-        idx_h.copy_(out_idx, non_blocking=True)
-
-    ms_e2e = timed(e2e_step, max(3, args.steps // 2), 2)
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, w_h, k_h, pos_h))
-    d2h = idx_h.numel() * idx_h.element_size()
-
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):
         with open(tfile) as f:
             traffic = json.load(f).get(wl.name, {}).get("score_tc_kernel")
-    # the kernel's bound is whichever of its algorithmic flops and bytes takes longer at peak
-    flops = algorithmic_flops_score(wl)
-    score_bytes = algorithmic_bytes_score(wl)
-    form = "block form" if block_form(wl) else "decode form"
-    if flops / (peaks["bf16"] * 1e12) > score_bytes / (peaks["hbm"] * 1e9):
-        achieved = flops / (ms_score_kernel * 1e-3) / 1e12
-        roofline = {"kernel": f"score_tc_kernel (routed scoring, {form})", "bound": "tensor",
-                    "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16"], "traffic": traffic,
-                    "peak_source": peaks["source"] + " bf16 dense (burst)",
-                    "algorithmic_flops": flops, "algorithmic_bytes": score_bytes,
-                    "avg_ms": ms_score_kernel}
-    else:
-        achieved = score_bytes / (ms_score_kernel * 1e-3) / 1e9
-        roofline = {"kernel": f"score_tc_kernel (routed scoring, {form})", "bound": "hbm",
-                    "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm"], "traffic": traffic,
-                    "peak_source": peaks["source"] + " HBM copy",
-                    "algorithmic_bytes": score_bytes, "algorithmic_flops": flops,
-                    "avg_ms": ms_score_kernel}
-
-    launches_per_step = misa_step_launches(wl)
-    if ms_kept is not None:
-        kept = {"value": units * world / (ms_kept * 1e-3), "ms_per_step": ms_kept,
-                "speedup_vs_dsa": ms_dsa / ms_kept,
-                "step": "refresh the newest key's pooled block + route + routed score + top-k"}
-    line = {
-        "metric": METRIC, "value": units * world / (ms_misa * 1e-3), "unit": UNIT,
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_misa,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
+    res = {
+        "value": units * world / (ms_misa * 1e-3), "unit": UNIT, "ms_per_step": ms_misa,
         "config": {"workload": wl.name, "nseq": nseq, "T": T, "L": wl.L, "H": H, "d": d,
-                   "h": wl.h, "B": wl.B, "topk": wl.topk, "kprime": wl.kprime,
-                   "path": "MISA: pool + route + routed score + top-k",
-                   "l2": "inputs > L2 (keys %.0f MB), two resident copies used alternately"
-                         % (x.k_bits.nbytes / 1e6),
-                   "parallelism": "replicas" if world > 1 else "single"},
-        "roofline": roofline,
+                   "h": wl.h, "B": wl.B, "topk": wl.topk, "kprime": wl.kprime},
+        "roofline": _roofline(wl, ms_score_kernel, peaks, traffic),
         "paths": {
             "misa": {"value": units * world / (ms_misa * 1e-3), "ms_per_step": ms_misa,
                      "ms_pool": call_ms[0], "ms_route": call_ms[1], "ms_score_topk": call_ms[2],
                      "ms_score_kernel_alone": ms_score_kernel},
             "dsa": {"value": units * world / (ms_dsa * 1e-3), "ms_per_step": ms_dsa},
-            "misa_dagger": {"value": units * world / (ms_dagger * 1e-3), "ms_per_step": ms_dagger},
+            "misa_dagger": {"value": units * world / (ms_dagger * 1e-3),
+                            "ms_per_step": ms_dagger},
             "speedup_misa_vs_dsa": ms_dsa / ms_misa,
             "speedup_dagger_vs_dsa": ms_dsa / ms_dagger,
             "recall_vs_dsa": recalls,
         },
-        "e2e": {"value": units * world / (ms_e2e * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "l2": "inputs > L2 (keys %.0f MB, q %.0f MB), two resident copies used alternately"
+              % (x.k_bits.nbytes / 1e6, x.q_bits.nbytes / 1e6),
     }
+    if not decode and wl.kprime >= int(np.mean(x.pos)) + 1:
+        res["paths"]["misa_dagger"]["note"] = (
+            f"k'={wl.kprime} is at least the mean causal prefix: the re-rank re-scores about "
+            "every prefix token with all heads (MISA-dagger is a decode method)")
+    if ms_hisa is not None:
+        res["paths"]["hisa_block_filter"] = {
+            "value": units * world / (ms_hisa * 1e-3), "ms_per_step": ms_hisa,
+            "speedup_vs_dsa": ms_dsa / ms_hisa, "B": hisa_B, "m": hisa_m,
+            "step": "pool (B=128) + head-summed block scores + top-m blocks + all-head "
+                    "re-score of their tokens + top-k"}
     if ms_kept is not None:
-        line["paths"]["misa_kept_pool"] = kept
+        res["paths"]["misa_kept_pool"] = {
+            "value": units * world / (ms_kept * 1e-3), "ms_per_step": ms_kept,
+            "speedup_vs_dsa": ms_dsa / ms_kept,
+            "step": "refresh the newest key's pooled block + route + routed score + top-k"}
+
+    if headline:
+        # end to end through the public API: pinned host inputs -> device -> MISA -> host
+        idx_h = torch.empty((nseq, T, wl.topk), dtype=torch.int32).pin_memory()
+        e2e_dev = [torch.empty_like(t) for t in sets[0]]
+
+        def e2e_step(i):
+            for dst, src in zip(e2e_dev, (q_h, w_h, k_h, pos_h)):
+                dst.view(src.dtype).copy_(src, non_blocking=True)
+            q, w, k, pos = e2e_dev
+            out_idx, _, _ = M.misa_indexer(q, w, k, pos, wl.B, wl.h, wl.topk)
+            idx_h.copy_(out_idx, non_blocking=True)
+
+        ms_e2e = timed(e2e_step, max(3, args.steps // 2), 3)
+        h2d = sum(t.numel() * t.element_size() for t in (q_h, w_h, k_h, pos_h))
+        d2h = idx_h.numel() * idx_h.element_size()
+        res["e2e"] = {"value": units * world / (ms_e2e * 1e-3), "unit": UNIT,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del sets, kp
+    torch.cuda.empty_cache()
+    return res, ms_misa
+
+
+def run_cuda(args, wl):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=dev)
+    import long_context_block_b200 as M
+    peaks = _peaks()
+
+    head, ms_misa = measure_workload(M, wl, args, dev, world, rank, peaks, headline=True)
+    if args.only:
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(head))
+        return 0
+    extra = {}
+    if args.all_configs and wl.name == DEFAULT_WORKLOAD:
+        for name in EXTRA_WORKLOADS:   # the other configs of the metric, same steps
+            r, _ = measure_workload(M, WORKLOADS[name], args, dev, world, rank, peaks,
+                                    headline=False)
+            extra[name] = r
+
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_misa,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(head["config"], path="MISA: pool + route + routed score + top-k",
+                       l2=head["l2"], parallelism="replicas" if world > 1 else "single"),
+        "roofline": head["roofline"],
+        "paths": head["paths"],
+        "e2e": head["e2e"],
+        "gpu_launches": misa_step_launches(wl) * args.steps,
+        "clocks": head["clocks"],
+    }
+    if extra:
+        line["configs"] = extra
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -497,7 +570,11 @@ def main():
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override an integer field of the workload (e.g. T=8192), for "
                          "smaller profiling runs; the JSON line names the result")
-    ap.add_argument("--only", choices=["misa", "dagger", "dsa"],
+    ap.add_argument("--no-all-configs", dest="all_configs", action="store_false",
+                    help="time only the headline workload (by default the 32K decode run also "
+                         "times the 16K prefill, GLM-5 128K and MISA-dagger 128K workloads "
+                         "and reports them under 'configs')")
+    ap.add_argument("--only", choices=["misa", "dagger", "dsa", "kept", "hisa"],
                     help="run only this path's warm-up + timed steps, untimed, and print no "
                          "bench line (for profiler captures)")
     args = ap.parse_args()

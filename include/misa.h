@@ -71,11 +71,12 @@ extern "C" {
 #define MISA_OP_DSA_TOPK      3
 #define MISA_OP_DAGGER_RERANK 4
 #define MISA_OP_SCORE_ROWS    5
+#define MISA_OP_HISA_TOPK     6
 
 /* Limits of this build (larger values return MISA_ERR_UNSUPPORTED). */
 #define MISA_HEAD_DIM        128
 #define MISA_MAX_HEADS       128
-#define MISA_MAX_ROUTED      16
+#define MISA_MAX_ROUTED      128  /* h <= H <= MISA_MAX_HEADS */
 #define MISA_MAX_TOPK        16384
 
 /*
@@ -172,6 +173,25 @@ int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k,
                        void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * HISA-style token-axis block filter, the variant the pages contrast MISA with
+ * ("Key distinction from HISA", Methodology section 1; the HISA abstract's
+ * block-level coarse filter followed by token-level refinement).  Both use the
+ * router's affinities A[j, b] = w[j] * ReLU(q[j] . kp_b) over the blocks of the
+ * query's prefix (partial last block as in misa_route_heads); this one reduces
+ * them across heads, G[b] = sum_j A[j, b], keeps the m blocks with the largest G
+ * (ties: lower b), scores the tokens of the kept blocks with all H heads (Eq. 1),
+ * and returns their topk best in idx / vals (order and padding as elsewhere).
+ * k_pool must hold the pooled keys for this B (misa_pool_keys).  blocks (nullable,
+ * int32 [nseq, T, m]) receives the kept blocks by descending G, -1 padded.
+ * 1 <= m, m * B <= MISA_MAX_TOPK.
+ * Needs misa_workspace_size(MISA_OP_HISA_TOPK, ..., B, m (as h), topk, 0).
+ */
+int hisa_block_filter_topk(const uint16_t* q, const float* w, const uint16_t* k,
+                           const float* k_pool, const int32_t* pos, int nseq, int T, int H,
+                           int d, int64_t L, int B, int m, int topk, int32_t* idx, float* vals,
+                           int32_t* blocks, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * misa_score_topk without any allocation or workspace.  The paper has no
  * counterpart of this entry point; it serves callers that cannot allocate device
  * memory or pass a workspace (code running inside an allocator-free region of a
@@ -184,8 +204,10 @@ int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k,
  * MISA_ERR_STATIC_SCRATCH_TOO_SMALL and enqueue nothing.  All calls on a device
  * share that array and it keeps the last call's contents, so calls whose GPU work
  * overlaps (other streams, other host threads) race and must be serialised by the
- * caller.  The first call on each device looks up the array's address with that
- * device current; make it before any stream capture.  device_status (nullable,
+ * caller.  Every call looks up the array's address with the caller's device
+ * current; the first call on a device also loads the library there, so make it
+ * before any stream capture.  Pointers are checked like misa_score_topk's (on the
+ * current device, aligned, long enough); a bad one returns MISA_ERR_INVALID_ARG.  device_status (nullable,
  * device int32) receives this call's device-side status word (MISA_OK or
  * MISA_ERR_BAD_DEVICE_INPUT), as misa_check_device_status would report it.
  * Calls no cudaMalloc, cudaFree or allocating library routine.

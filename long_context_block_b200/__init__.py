@@ -5,6 +5,7 @@ binding plus two compositions of the entry points:
 
   misa_indexer  -- pool keys, route heads, routed score + top-k   (Eqs. 4, 7-10)
   misa_dagger   -- misa_indexer with k' candidates, then the all-head re-rank (Eqs. 11-12)
+  hisa_indexer  -- the HISA-style token-axis block filter the pages contrast MISA with
 
 Reference: "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
 Inference" (picx.dev summary page, Methodology sections 1-2).
@@ -16,6 +17,7 @@ from ._binding import (  # noqa: F401
     MisaError,
     declared_symbols,
     dsa_score_topk,
+    hisa_block_filter_topk,
     library,
     misa_check_device_status,
     misa_dagger_rerank,
@@ -25,6 +27,8 @@ from ._binding import (  # noqa: F401
     misa_score_rows,
     misa_score_topk,
     misa_score_topk_noalloc,
+    misa_testing_score_rows_wait_expiry,
+    misa_testing_score_simt,
     misa_workspace_size,
     workspace,
 )
@@ -52,3 +56,12 @@ def misa_dagger(q, w, k, pos, B: int, h: int, topk: int, kprime: int, k_pool=Non
     cand = misa_score_topk(q, w, k, heads, pos, kprime, return_vals=False)
     idx, vals = misa_dagger_rerank(q, w, k, pos, cand, topk)
     return idx, vals, cand, heads
+
+
+def hisa_indexer(q, w, k, pos, B: int, m: int, topk: int, k_pool=None):
+    """HISA-style block filter: pool with B (skipped when k_pool is given), keep each
+    query's top-m blocks by head-summed affinity, top-k of the all-head scores of their
+    tokens.  Returns (idx, vals, blocks)."""
+    if k_pool is None:
+        k_pool = misa_pool_keys(k, B)
+    return hisa_block_filter_topk(q, w, k, k_pool, pos, B, m, topk, return_blocks=True)

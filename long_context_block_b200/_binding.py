@@ -18,7 +18,8 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmisa_b200.so")
-HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "misa.h")
+INCLUDE_DIR = os.path.join(os.path.dirname(_PKG), "include")
+HEADER_PATH = os.path.join(INCLUDE_DIR, "misa.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -47,6 +48,14 @@ _SIGS = {
                                  _c_int, _p, _p, _c_sz, _p]),
     "misa_score_topk_noalloc": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
                                          _c_i64, _c_int, _c_int, _p, _p, _p, _p]),
+    "hisa_block_filter_topk": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int, _c_int,
+                                        _c_i64, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_sz,
+                                        _p]),
+    "misa_testing_score_simt": (_c_int, [_p, _p, _p, _p, _p, _p, _p, _c_int, _c_int, _c_int,
+                                         _c_int, _c_i64, _c_int, _c_i64, _p, _p, _c_sz, _p]),
+    "misa_testing_score_rows_wait_expiry": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int,
+                                                     _c_int, _c_i64, _c_int, _p, _p, _c_sz,
+                                                     ctypes.c_longlong, _c_int, _p]),
     "misa_status_string": (ctypes.c_char_p, [_c_int]),
     "misa_check_device_status": (_c_int, [_p, _p]),
 }
@@ -55,6 +64,7 @@ for _name, (_res, _args) in _SIGS.items():
     _f.restype, _f.argtypes = _res, _args
 
 OP_ROUTE_HEADS, OP_SCORE_TOPK, OP_DSA_TOPK, OP_DAGGER_RERANK, OP_SCORE_ROWS = 1, 2, 3, 4, 5
+OP_HISA_TOPK = 6
 HEAD_DIM = 128
 
 
@@ -65,11 +75,15 @@ class MisaError(RuntimeError):
 
 
 def declared_symbols() -> list[str]:
-    """Function names declared in include/misa.h."""
-    text = open(HEADER_PATH).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) -
-                  {"if", "sizeof", "defined"})
+    """Function names declared in the headers under include/ (misa.h and misa_testing.h)."""
+    names = set()
+    for f in sorted(os.listdir(INCLUDE_DIR)):
+        if not f.endswith(".h"):
+            continue
+        text = open(os.path.join(INCLUDE_DIR, f)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text))
+    return sorted(names - {"if", "sizeof", "defined"})
 
 
 def library() -> ctypes.CDLL:
@@ -298,6 +312,35 @@ def misa_dagger_rerank(q, w, k, pos, cand, topk: int, return_vals: bool = True, 
     return (idx, vals) if return_vals else idx
 
 
+def hisa_block_filter_topk(q, w, k, k_pool, pos, B: int, m: int, topk: int,
+                           return_vals: bool = True, return_blocks: bool = False, idx=None,
+                           vals=None, blocks=None):
+    """HISA-style token-axis filter: keep each query's m blocks with the largest
+    head-summed affinity G[b] = sum_j w_j ReLU(q_j . kp_b), then the top-k of the
+    all-head score (Eq. 1) over their tokens.  k_pool: misa_pool_keys(k, B)."""
+    q, k = _bits(q, "q"), _bits(k, "k")
+    w = _dev(w, "w", torch.float32)
+    k_pool = _dev(k_pool, "k_pool", torch.float32)
+    pos = _dev(pos, "pos", torch.int32)
+    nseq, T, H, d = q.shape
+    L = k.shape[1]
+    idx, vals = _outs((nseq, T), topk, q.device, idx, vals, return_vals)
+    if return_blocks and blocks is None:
+        blocks = torch.empty((nseq, T, m), dtype=torch.int32, device=q.device)
+    nb = misa_workspace_size(OP_HISA_TOPK, nseq, T, H, d, L, B, m, topk, 0)
+    if nb == 0:
+        raise MisaError("misa_workspace_size", 1)
+    ws = _WS.get(nb, q.device)
+    _check("hisa_block_filter_topk",
+           _lib.hisa_block_filter_topk(_ptr(q), _ptr(w), _ptr(k), _ptr(k_pool), _ptr(pos), nseq,
+                                       T, H, d, L, B, m, topk, _ptr(idx), _ptr(vals),
+                                       _ptr(blocks), _ptr(ws), ws.numel(), _stream()))
+    out = (idx, vals) if return_vals else (idx,)
+    if return_blocks:
+        out = out + (blocks,)
+    return out if len(out) > 1 else out[0]
+
+
 def misa_score_topk_noalloc(q, w, k, heads, pos, topk: int, return_vals: bool = True, idx=None,
                             vals=None, device_status=None):
     """misa_score_topk for callers that cannot allocate: the library uses its own fixed
@@ -318,3 +361,63 @@ def misa_score_topk_noalloc(q, w, k, heads, pos, topk: int, return_vals: bool = 
                                         T, H, d, L, h, topk, _ptr(idx), _ptr(vals),
                                         _ptr(device_status), _stream()))
     return (idx, vals) if return_vals else idx
+
+
+# ----------------------------------------------------------------- test-only entry points
+# (include/misa_testing.h): the CUDA-core scorer on its own, and the tensor-core scorer
+# with shortened wait bounds and one key tile never loaded.
+
+def misa_testing_score_simt(q, w, k, heads, pos, gather_ids=None, gather_len=None,
+                            scores: torch.Tensor | None = None):
+    """The CUDA-core scorer: Eq. (9) under heads (Eq. 1 with heads None) over each
+    query's prefix, or over gather_ids[row, :gather_len[row]] when given.  Returns fp32
+    [nseq, T, L] (prefix) or [nseq, T, kprime] (gather)."""
+    q, k = _bits(q, "q"), _bits(k, "k")
+    w = _dev(w, "w", torch.float32)
+    pos = _dev(pos, "pos", torch.int32)
+    nseq, T, H, d = q.shape
+    L = k.shape[1]
+    if heads is not None:
+        heads = _dev(heads, "heads", torch.int32)
+    h = heads.shape[-1] if heads is not None else H
+    if gather_ids is not None:
+        gather_ids = _dev(gather_ids, "gather_ids", torch.int32)
+        gather_len = _dev(gather_len, "gather_len", torch.int32)
+        stride = gather_ids.shape[-1]
+    else:
+        stride = L
+    if scores is None:
+        scores = torch.full((nseq, T, stride), float("nan"), dtype=torch.float32,
+                            device=q.device)
+    ws = _WS.get(256, q.device)
+    _check("misa_testing_score_simt",
+           _lib.misa_testing_score_simt(_ptr(q), _ptr(w), _ptr(k), _ptr(heads), _ptr(pos),
+                                        _ptr(gather_ids), _ptr(gather_len), nseq, T, H, d, L, h,
+                                        stride, _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    return scores
+
+
+def misa_testing_score_rows_wait_expiry(q, w, k, heads, pos, wait_cycles: int, skip_tile: int,
+                                        scores: torch.Tensor | None = None):
+    """misa_score_rows with every wait bounded by wait_cycles and key tile skip_tile never
+    loaded (-1: none).  Read the outcome with misa_check_device_status."""
+    q, k = _bits(q, "q"), _bits(k, "k")
+    w = _dev(w, "w", torch.float32)
+    pos = _dev(pos, "pos", torch.int32)
+    nseq, T, H, d = q.shape
+    L = k.shape[1]
+    if heads is not None:
+        heads = _dev(heads, "heads", torch.int32)
+    h = heads.shape[-1] if heads is not None else H
+    if scores is None:
+        scores = torch.full((nseq, T, L), float("nan"), dtype=torch.float32, device=q.device)
+    nb = misa_workspace_size(OP_SCORE_ROWS, nseq, T, H, d, L, 1, h, 1, 1)
+    if nb == 0:
+        raise MisaError("misa_workspace_size", 1)
+    ws = _WS.get(nb, q.device)
+    _check("misa_testing_score_rows_wait_expiry",
+           _lib.misa_testing_score_rows_wait_expiry(_ptr(q), _ptr(w), _ptr(k), _ptr(heads),
+                                                    _ptr(pos), nseq, T, H, d, L, h,
+                                                    _ptr(scores), _ptr(ws), ws.numel(),
+                                                    int(wait_cycles), int(skip_tile), _stream()))
+    return scores

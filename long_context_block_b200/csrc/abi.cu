@@ -9,54 +9,11 @@
 
 #include "internal.h"
 #include "misa.h"
+#include "misa_testing.h"
 
 using namespace misa;
 
 namespace {
-
-using GetRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
-
-GetRangeFn get_range_fn() {
-  static GetRangeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<GetRangeFn>(p);
-    cudaGetLastError();
-  });
-  return fn;
-}
-
-// A device buffer of at least `bytes` bytes, `align`-aligned, allocated on a CUDA device.
-int check_dev(const void* p, size_t bytes, size_t align) {
-  if (p == nullptr) return MISA_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(p) % align) return MISA_ERR_INVALID_ARG;
-  cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-    cudaGetLastError();
-    return MISA_ERR_INVALID_ARG;
-  }
-  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
-    return MISA_ERR_INVALID_ARG;
-  if (a.type == cudaMemoryTypeDevice) {
-    if (GetRangeFn fn = get_range_fn()) {
-      CUdeviceptr base = 0;
-      size_t size = 0;
-      if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(p)) == CUDA_SUCCESS) {
-        if (reinterpret_cast<uintptr_t>(p) + bytes > (uintptr_t)base + size)
-          return MISA_ERR_INVALID_ARG;
-      }
-    }
-  }
-  return MISA_OK;
-}
-int check_opt(const void* p, size_t bytes, size_t align) {
-  return p == nullptr ? MISA_OK : check_dev(p, bytes, align);
-}
 
 #define MISA_TRY(expr)            \
   do {                            \
@@ -140,6 +97,10 @@ size_t misa_workspace_size(int op, int nseq, int T, int H, int d, int64_t L, int
     case MISA_OP_DAGGER_RERANK:
       if (check_topk(topk) != MISA_OK || kprime < topk || kprime > MISA_MAX_TOPK) return 0;
       return dagger_ws(nseq, T, H, kprime);
+    case MISA_OP_HISA_TOPK:   // h carries m
+      if (B < 1 || h < 1 || (int64_t)h * B > MISA_MAX_TOPK || check_topk(topk) != MISA_OK)
+        return 0;
+      return kStatusBytes + hisa_ws_bytes(nseq, T, H, L, B, h);
     default:
       return 0;
   }
@@ -319,6 +280,29 @@ int misa_dagger_rerank(const uint16_t* q, const float* w, const uint16_t* k, con
                                  vals, status, st));
 }
 
+int hisa_block_filter_topk(const uint16_t* q, const float* w, const uint16_t* k,
+                           const float* k_pool, const int32_t* pos, int nseq, int T, int H, int d,
+                           int64_t L, int B, int m, int topk, int32_t* idx, float* vals,
+                           int32_t* blocks, void* ws, size_t ws_bytes, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  MISA_TRY(check_topk(topk));
+  if (B < 1 || m < 1) return MISA_ERR_INVALID_ARG;
+  if ((int64_t)m * B > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)nseq * T;
+  const int64_t M = (L + B - 1) / B;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(k_pool, (size_t)nseq * M * d * 4, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  MISA_TRY(check_dev(idx, rows * topk * 4, 4));
+  MISA_TRY(check_opt(vals, rows * topk * 4, 4));
+  MISA_TRY(check_opt(blocks, rows * m * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, kStatusBytes + hisa_ws_bytes(nseq, T, H, L, B, m)));
+  return cuda_status(launch_hisa(q, w, k, k_pool, pos, nseq, T, H, L, B, m, topk, idx, vals,
+                                 blocks, ws_region(ws, 0), status_word(ws), (cudaStream_t)stream));
+}
+
 const char* misa_status_string(int status) {
   switch (status) {
     case MISA_OK: return "ok";
@@ -342,6 +326,64 @@ int misa_check_device_status(void* ws, void* stream) {
   if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MISA_ERR_CUDA;
   if (v != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MISA_ERR_CUDA;
   return v;
+}
+
+// ---------------------------------------------------------------- test-only entry points
+// (declared in include/misa_testing.h)
+
+int misa_testing_score_simt(const uint16_t* q, const float* w, const uint16_t* k,
+                            const int32_t* heads, const int32_t* pos, const int32_t* gather_ids,
+                            const int32_t* gather_len, int nseq, int T, int H, int d, int64_t L,
+                            int h, int64_t out_stride, float* scores, void* ws, size_t ws_bytes,
+                            void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  if (h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  const bool gather = gather_ids != nullptr;
+  if (gather != (gather_len != nullptr)) return MISA_ERR_INVALID_ARG;
+  if (out_stride < 1 || (!gather && out_stride < L) || out_stride >= INT32_MAX)
+    return MISA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)nseq * T;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  if (heads) MISA_TRY(check_dev(heads, rows * h * 4, 4));
+  if (gather) {
+    MISA_TRY(check_dev(gather_ids, rows * out_stride * 4, 4));
+    MISA_TRY(check_dev(gather_len, rows * 4, 4));
+  }
+  MISA_TRY(check_dev(scores, rows * out_stride * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+  return cuda_status(launch_score_simt(q, w, k, heads, h, pos, gather_ids, gather_len, nseq, T,
+                                       H, L, scores, out_stride, status_word(ws),
+                                       (cudaStream_t)stream));
+}
+
+int misa_testing_score_rows_wait_expiry(const uint16_t* q, const float* w, const uint16_t* k,
+                                        const int32_t* heads, const int32_t* pos, int nseq,
+                                        int T, int H, int d, int64_t L, int h, float* scores,
+                                        void* ws, size_t ws_bytes, long long wait_cycles,
+                                        int skip_tile, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  if (h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  if (wait_cycles < 1000 || wait_cycles > 4000000000LL || skip_tile < -1)
+    return MISA_ERR_INVALID_ARG;
+  const int nh = heads ? h : H;
+  if (!score_tc_supported(nseq, T, nh, L)) return MISA_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)nseq * T;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  if (heads) MISA_TRY(check_dev(heads, rows * h * 4, 4));
+  MISA_TRY(check_dev(scores, rows * L * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, kStatusBytes + score_tc_ws_bytes(nseq, T, nh)));
+  WaitProbe probe;
+  probe.wait_cycles = wait_cycles;
+  probe.skip_tile = skip_tile;
+  return cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, scores, L,
+                                     ws_region(ws, 0), status_word(ws), nullptr,
+                                     (cudaStream_t)stream, nullptr, nullptr, &probe));
 }
 
 }  // extern "C"

@@ -27,6 +27,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Host checks of a caller's device buffer (validate.cu): non-null, `align`-aligned, on the
+// current device, and at least `bytes` long when its allocation range can be queried.
+// Return MISA_OK or MISA_ERR_INVALID_ARG.  check_opt accepts a null pointer.
+int check_dev(const void* p, size_t bytes, size_t align);
+int check_opt(const void* p, size_t bytes, size_t align);
+
 // Workspace layout helpers: every region starts on a 256-byte boundary.
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -54,6 +60,22 @@ cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
                          const float* k_pool, const int32_t* pos, int nseq, int T, int H,
                          int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
                          int nchunk, int* counters, int* status, cudaStream_t st);
+
+// K2 in block-score mode (route.cu), for the HISA-style filter: G[row, b] = sum_j
+// w[row,j] * ReLU(q[row,j] . kp_b) for the blocks b < M_t of each query's prefix (row stride
+// ceil(L/B)), and last_block[row] = M_t - 1.
+cudaError_t launch_block_scores(const uint16_t* q, const float* w, const uint16_t* k,
+                                const float* k_pool, const int32_t* pos, int nseq, int T, int H,
+                                int64_t L, int B, float* G, int32_t* last_block, int* status,
+                                cudaStream_t st);
+
+// K8 -- the HISA-style token-axis block filter (hisa.cu): block scores, top-m blocks, their
+// tokens re-scored with all H heads, top-k.  Scratch: hisa_ws_bytes(...), 256-aligned.
+size_t hisa_ws_bytes(int nseq, int T, int H, int64_t L, int B, int m);
+cudaError_t launch_hisa(const uint16_t* q, const float* w, const uint16_t* k, const float* k_pool,
+                        const int32_t* pos, int nseq, int T, int H, int64_t L, int B, int m,
+                        int topk, int32_t* idx, float* vals, int32_t* blocks, void* scratch,
+                        int* status, cudaStream_t st);
 
 // K2 -- router on tcgen05 for sequences with many queries (route_tc.cu): the full-block
 // part of Eq. (7) as a GEMM against the sequence's pooled keys (bf16 hi + lo), the partial
@@ -88,12 +110,21 @@ size_t score_tc_ws_bytes(int nseq, int T, int nh, bool gather = false);
 //   gather_ids / gather_len (both or neither): row r scores the gather_len[r] tokens
 //   gather_ids[r * out_stride + i] (each in [0, L)) into out[r * out_stride + i]; every
 //   row takes the decode form and its keys are fetched four rows per TMA gather.
+//   test_probe (nullable; tests only): a shorter bound for every wait of the scorer and
+//   one key tile (global index in the CTAs' end-to-end tile order) that is never loaded,
+//   so that a wait runs out and the expiry path (record MISA_ERR_DEVICE_TIMEOUT, let the
+//   copies and MMAs in flight finish, free TMEM, return) runs.
+struct WaitProbe {
+  long long wait_cycles;
+  int skip_tile;
+};
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
                             int* status, uint32_t* hist, cudaStream_t st,
                             const int32_t* gather_ids = nullptr,
-                            const int32_t* gather_len = nullptr);
+                            const int32_t* gather_len = nullptr,
+                            const WaitProbe* test_probe = nullptr);
 
 // K5 -- per-row top-k selection (topk.cu).
 //   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.

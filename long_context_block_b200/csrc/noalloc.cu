@@ -16,13 +16,12 @@
 //  * Every call on a device uses the same array, and the array keeps what the last
 //    call left in it.  Calls whose GPU work overlaps (different streams, or several
 //    host threads) race on it and must be serialised by the caller.
-//  * The first call on each device looks up the array's device address
-//    (cudaGetSymbolAddress) with that device current; make that first call before
-//    any stream capture.
+//  * Every call looks up the array's device address (cudaGetSymbolAddress) with the
+//    caller's device current; the first call on a device also loads the library's
+//    device image there, so make that first call before any stream capture.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "internal.h"
 #include "misa.h"
@@ -31,38 +30,19 @@ namespace {
 
 constexpr size_t kNoAllocScoreCapacity = size_t(4) << 20;   // fp32 scores (16 MiB)
 constexpr size_t kNoAllocBytes = misa::kStatusBytes + kNoAllocScoreCapacity * sizeof(float);
-constexpr int kMaxDevices = 64;
-
 // Scratch of the no-allocation entry point: status word (first 256 bytes), then scores.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array on the current device.  Looked up on every call (it
+// allocates nothing), so the address is never stale, e.g. after a cudaDeviceReset.
 int scratch_for_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MISA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return MISA_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return MISA_OK;
-}
-
-bool is_device_ptr(const void* p) {
-  cudaPointerAttributes a;
-  if (p == nullptr || cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
     cudaGetLastError();
-    return false;
+    return MISA_ERR_CUDA;
   }
-  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+  *out = p;
+  return MISA_OK;
 }
 
 }  // namespace
@@ -75,22 +55,25 @@ extern "C" int misa_score_topk_noalloc(const uint16_t* q, const float* w, const 
   if (d != MISA_HEAD_DIM || H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
   if (h < 1 || h > H || topk < 1) return MISA_ERR_INVALID_ARG;
   if (h > MISA_MAX_ROUTED || topk > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
-  if (q == nullptr || w == nullptr || k == nullptr || heads == nullptr || pos == nullptr ||
-      idx == nullptr)
-    return MISA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k)) % 16)
-    return MISA_ERR_INVALID_ARG;
   const size_t rows = (size_t)nseq * T;
   if (rows * (size_t)L > kNoAllocScoreCapacity) return MISA_ERR_STATIC_SCRATCH_TOO_SMALL;
-  for (const void* p : {(const void*)q, (const void*)w, (const void*)k, (const void*)heads,
-                        (const void*)pos, (const void*)idx})
-    if (!is_device_ptr(p)) return MISA_ERR_INVALID_ARG;
-  if ((vals && !is_device_ptr(vals)) || (device_status && !is_device_ptr(device_status)))
-    return MISA_ERR_INVALID_ARG;
+  // the same buffer checks as misa_score_topk: every pointer on the current device,
+  // aligned, and long enough for what the kernels read and write
+  using misa::check_dev;
+  using misa::check_opt;
+  int s = MISA_OK;
+  if ((s = check_dev(q, rows * H * d * 2, 16)) != MISA_OK ||
+      (s = check_dev(w, rows * H * 4, 4)) != MISA_OK ||
+      (s = check_dev(k, (size_t)nseq * L * d * 2, 16)) != MISA_OK ||
+      (s = check_dev(heads, rows * h * 4, 4)) != MISA_OK ||
+      (s = check_dev(pos, rows * 4, 4)) != MISA_OK ||
+      (s = check_dev(idx, rows * topk * 4, 4)) != MISA_OK ||
+      (s = check_opt(vals, rows * topk * 4, 4)) != MISA_OK ||
+      (s = check_opt(device_status, 4, 4)) != MISA_OK)
+    return s;
 
   void* scratch = nullptr;
-  const int s = scratch_for_current_device(&scratch);
-  if (s != MISA_OK) return s;
+  if ((s = scratch_for_current_device(&scratch)) != MISA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   int* status = reinterpret_cast<int*>(scratch);
   float* scores = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + misa::kStatusBytes);

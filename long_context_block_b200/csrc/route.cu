@@ -16,6 +16,11 @@
 // the last CTA of a row to finish sums the chunk partials, applies |w_j| / M_t (common
 // to all blocks, so applied once), writes E and selects the top-h heads by repeated
 // warp arg-max.
+//
+// The same kernel, in its block-score mode, reduces the affinities along the other axis
+// for the HISA-style token-axis filter (MISA page, "Key distinction from HISA"):
+// G[t,b] = sum_j A[t,j,b] = sum_j w[t,j] * ReLU(q[t,j] . kp_b), one value per block of
+// the query's prefix, written straight to G (each CTA owns its chunk's blocks).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -87,7 +92,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int MT>   // 16-head row tiles per warp (ceil(ceil(H/16) / 4))
+// kBlockScores: write G[row, b] = sum_j w_j * ReLU(q_j . kp_b) for the chunk's blocks to
+// `partial` (row stride Mpool) and M_t - 1 to counters[row] (the last block index), instead
+// of the head energies.
+template <int MT, bool kBlockScores>   // MT: 16-head row tiles per warp (ceil(ceil(H/16)/4))
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
     const float* __restrict__ k_pool, const int32_t* __restrict__ pos, int T, int H,
@@ -115,6 +123,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   const int nb = min(b0 + kCh, M) - b0;
   const int64_t n = row / T;
   const bool has_part = Mfull < M && Mfull >= b0 && Mfull < b0 + nb;
+  if (kBlockScores && chunk == 0 && tid == 0) counters[row] = M - 1;
 
   // the partial last block of this prefix: mean of keys Mfull*B .. P-1 (fp32)
   if (has_part) {
@@ -212,6 +221,41 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
       }
     }
   }
+  if constexpr (kBlockScores) {
+    // G[b] = sum_j w_j * ReLU(S[j, b]): this thread's heads (rows g, g + 8 of each of its
+    // tiles), then the 8 lanes sharing its columns, then the 4 warps
+    float gs[kNT][2];
+#pragma unroll
+    for (int t = 0; t < kNT; ++t) gs[t][0] = gs[t][1] = 0.f;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const int r0 = (warp + 4 * m) * 16;
+      const float wa = r0 + g < H ? w[row * H + r0 + g] : 0.f;
+      const float wb = r0 + g + 8 < H ? w[row * H + r0 + g + 8] : 0.f;
+#pragma unroll
+      for (int t = 0; t < kNT; ++t)
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          gs[t][i] += wa * fmaxf(acc[m][t][i], 0.f) + wb * fmaxf(acc[m][t][2 + i], 0.f);
+    }
+#pragma unroll
+    for (int t = 0; t < kNT; ++t)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float v = gs[t][i];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if (g == 0) red[warp][t * 8 + 2 * c4 + i] = v;
+      }
+    __syncthreads();
+    if (tid < nb) {
+      float v = 0.f;
+#pragma unroll
+      for (int wv = 0; wv < kRouteThreads / 32; ++wv) v += red[wv][tid];
+      partial[row * Mpool + b0 + tid] = v;
+    }
+  } else {
   // sum_b ReLU(q_j . kp_b) over the chunk's valid blocks, per head
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
@@ -268,23 +312,25 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
     }
   }
   if (tid < 32) select_top_h(ev, H, h, heads + row * h);
+  }   // energies (not kBlockScores)
 }
 
-template <int MT>
+template <int MT, bool kBlockScores>
 static cudaError_t launch_mt(const uint16_t* q, const float* w, const uint16_t* k,
                              const float* k_pool, const int32_t* pos, int rows, int T, int H,
                              int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
                              int nchunk, int* counters, int* status, cudaStream_t st) {
   const int Mpool = (int)((L + B - 1) / B);
   const size_t smem = (size_t)(16 * 4 * MT + 2 * kCh) * kRowPad * sizeof(uint16_t);
-  cudaError_t err = cudaFuncSetAttribute(route_kernel<MT>,
+  cudaError_t err = cudaFuncSetAttribute(route_kernel<MT, kBlockScores>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
     dim3 grid(nchunk, (unsigned)nr);
-    err = launch_pdl(route_kernel<MT>, grid, dim3(kRouteThreads), smem, st, q, k, k_pool, pos, T,
-                     H, L, B, Mpool, partial, nchunk, status, row0, w, h, counters, heads, E);
+    err = launch_pdl(route_kernel<MT, kBlockScores>, grid, dim3(kRouteThreads), smem, st, q, k,
+                     k_pool, pos, T, H, L, B, Mpool, partial, nchunk, status, row0, w, h,
+                     counters, heads, E);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
@@ -300,10 +346,24 @@ cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
   cudaError_t err = cudaMemsetAsync(counters, 0, (size_t)rows * sizeof(int), st);
   if (err != cudaSuccess) return err;
   if (H <= 64)
-    return launch_mt<1>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk,
-                        counters, status, st);
-  return launch_mt<2>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial, nchunk,
-                      counters, status, st);
+    return launch_mt<1, false>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial,
+                               nchunk, counters, status, st);
+  return launch_mt<2, false>(q, w, k, k_pool, pos, rows, T, H, L, B, h, heads, E, partial,
+                             nchunk, counters, status, st);
+}
+
+cudaError_t launch_block_scores(const uint16_t* q, const float* w, const uint16_t* k,
+                                const float* k_pool, const int32_t* pos, int nseq, int T, int H,
+                                int64_t L, int B, float* G, int32_t* last_block, int* status,
+                                cudaStream_t st) {
+  const int rows = nseq * T;
+  const int64_t M = (L + B - 1) / B;
+  const int nchunk = (int)((M + kRouteChunk - 1) / kRouteChunk);
+  if (H <= 64)
+    return launch_mt<1, true>(q, w, k, k_pool, pos, rows, T, H, L, B, 1, nullptr, nullptr, G,
+                              nchunk, last_block, status, st);
+  return launch_mt<2, true>(q, w, k, k_pool, pos, rows, T, H, L, B, 1, nullptr, nullptr, G,
+                            nchunk, last_block, status, st);
 }
 
 }  // namespace misa

@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kTile) score_simt_kernel(
   const bool gather = gather_ids != nullptr;
   int len;
   if (gather) {
-    len = gather_len[row];
+    len = (int)min((int64_t)max(gather_len[row], 0), out_stride);
   } else {
     len = prefix_len(pos, row, L, (blockIdx.x == 0 && tid == 0) ? status : nullptr);
   }
@@ -73,7 +73,11 @@ __global__ void __launch_bounds__(kTile) score_simt_kernel(
   for (int64_t tile = blockIdx.x; tile * kTile < len; tile += gridDim.x) {
     const int i = (int)(tile * kTile) + tid;
     if (i >= len) continue;
-    const int64_t s = gather ? (int64_t)gather_ids[row * out_stride + i] : (int64_t)i;
+    int64_t s = gather ? (int64_t)gather_ids[row * out_stride + i] : (int64_t)i;
+    if (s < 0 || s >= L) {   // a gathered id outside the sequence: reported, scored as key 0
+      set_status(status, MISA_ERR_BAD_DEVICE_INPUT);
+      s = 0;
+    }
     const uint4* kr = k + (n * L + s) * 16;
     float acc[NH];
 #pragma unroll

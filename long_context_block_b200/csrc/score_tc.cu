@@ -89,9 +89,10 @@ struct Cfg {
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
 
-// Unit segment of a CTA's tile range: unit u contributes its local tiles [a, b).
+// Unit segment of a CTA's tile range: unit u contributes its local tiles [a, b); its
+// first tile has the global index o.
 struct Seg {
-  int u, a, b;
+  int u, a, b, o;
 };
 
 __device__ __forceinline__ int find_unit(const int32_t* off, int units, int t) {
@@ -109,6 +110,7 @@ __device__ __forceinline__ bool next_seg(const int32_t* off, int units, int t0, 
   const int o0 = off[u], o1 = off[u + 1];
   if (o0 >= t1) return false;
   s.u = u;
+  s.o = o0;
   s.a = max(t0, o0) - o0;
   s.b = min(t1, o1) - o0;
   ++u;
@@ -117,16 +119,17 @@ __device__ __forceinline__ bool next_seg(const int32_t* off, int units, int t0, 
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, long long limit) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, kWaitCycles);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, limit);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // Bounded wait used while shutting down: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status,
+                                           long long limit) {
   volatile int never = 0;
-  mbar_wait(bar, parity, &never, status, kWaitCycles);
+  mbar_wait(bar, parity, &never, status, limit);
 }
 
 __device__ __forceinline__ void epi_bar(int nthreads) {
@@ -148,9 +151,12 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     const int32_t* __restrict__ tile_off, int units, Units geo, int64_t L,
     float* __restrict__ out, int64_t out_stride, int* status, uint32_t* __restrict__ hist,
     const int32_t* __restrict__ gidx, const int32_t* __restrict__ glen,
-    const uint16_t* __restrict__ kraw) {
+    const uint16_t* __restrict__ kraw, WaitProbe probe) {
   pdl_prologue();
   using C = Cfg<HS, QB>;
+  // bound of every wait (about 2 s normally; a test passes a short one together with a
+  // key tile that is never loaded, probe.skip_tile, to make a wait run out)
+  const long long kWait = probe.wait_cycles;
   constexpr int N = C::N;
   constexpr int kEpiThreads = 32 * C::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
         while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
           const int slot = qissued % C::kQBufs;
           if (!mbar_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status,
-                         kWaitCycles))
+                         kWait))
             break;
           uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
           mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
           tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
           const int wslot = qissued % C::kWBufs;
           if (!mbar_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status,
-                         kWaitCycles)) {
+                         kWait)) {
             ++qissued;
             break;
           }
@@ -240,9 +246,13 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
           for (int j = sg.a; j < sg.b; ++j) {
             const int s = issued % C::kStages;
             if (!mbar_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status,
-                           kWaitCycles)) {
+                           kWait)) {
               ok = false;
               break;
+            }
+            if (sg.o + j == probe.skip_tile) {   // test only: this tile is never loaded
+              ++issued;
+              continue;
             }
             uint8_t* kb = base + C::kStageBase + s * kKeyTileBytes;
             mbar_arrive_expect_tx(&full[s], kKeyTileBytes);
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
       bool ok = true;
       while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
         const int slot = qissued % C::kQBufs;
-        if (!warp_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status)) break;
+        if (!warp_wait(&qempty[slot], ((qissued / C::kQBufs) & 1) ^ 1, abort_flag, status, kWait)) break;
         uint8_t* qb = base + C::kQBase + slot * C::kQBytes;
         if (lane == 0) {
           mbar_arrive_expect_tx(&qfull[slot], C::kQBytes);
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
           tma_load_2d(qb + C::kQHalf, &tm_q, &qfull[slot], 64, sg.u * N);
         }
         const int wslot = qissued % C::kWBufs;
-        if (!warp_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status)) {
+        if (!warp_wait(&wempty[wslot], ((qissued / C::kWBufs) & 1) ^ 1, abort_flag, status, kWait)) {
           ++qissued;
           break;
         }
@@ -309,7 +319,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
 #pragma unroll
             for (int i = 0; i < 4; ++i) rq[d][i] = rq[d + 1][i];
           if (j + kIdAhead < sg.b) fetch_ids(j + kIdAhead, rq[kIdAhead - 1]);
-          if (!warp_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status)) {
+          if (!warp_wait(&empty[s], ((issued / C::kStages) & 1) ^ 1, abort_flag, status, kWait)) {
             ok = false;
             break;
           }
@@ -335,11 +345,11 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
     __syncthreads();   // (A) every role has left its loop
     if (lane == 0) {   // let this CTA's own copies land before the CTA exits
       for (int i = max(0, issued - C::kStages); i < issued; ++i)
-        drain_wait(&full[i % C::kStages], (i / C::kStages) & 1, status);
+        drain_wait(&full[i % C::kStages], (i / C::kStages) & 1, status, kWait);
       for (int i = max(0, qissued - C::kQBufs); i < qissued; ++i)
-        drain_wait(&qfull[i % C::kQBufs], (i / C::kQBufs) & 1, status);
+        drain_wait(&qfull[i % C::kQBufs], (i / C::kQBufs) & 1, status, kWait);
       for (int i = max(0, wissued - C::kWBufs); i < wissued; ++i)
-        drain_wait(&wfull[i % C::kWBufs], (i / C::kWBufs) & 1, status);
+        drain_wait(&wfull[i % C::kWBufs], (i / C::kWBufs) & 1, status, kWait);
     }
     __syncthreads();   // (B)
   } else if (warp == 1) {
@@ -353,14 +363,14 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
       bool ok = true;
       while (ok && next_seg(tile_off, units, t0, t1, u, sg)) {
         const int slot = seg % C::kQBufs;
-        if (!mbar_wait(&qfull[slot], (seg / C::kQBufs) & 1, abort_flag, status, kWaitCycles)) break;
+        if (!mbar_wait(&qfull[slot], (seg / C::kQBufs) & 1, abort_flag, status, kWait)) break;
         const uint32_t qaddr = smem0 + C::kQBase + slot * C::kQBytes;
         for (int j = sg.a; j < sg.b; ++j) {
           const int s = it % C::kStages;
           const int acc = acc_it % C::kAcc;
-          if (!mbar_wait(&full[s], (it / C::kStages) & 1, abort_flag, status, kWaitCycles) ||
+          if (!mbar_wait(&full[s], (it / C::kStages) & 1, abort_flag, status, kWait) ||
               !mbar_wait(&accempty[acc], ((acc_it / C::kAcc) & 1) ^ 1, abort_flag, status,
-                         kWaitCycles)) {
+                         kWait)) {
             ok = false;
             break;
           }
@@ -384,7 +394,7 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
         ++seg;
       }
       mma_commit(drain);   // completes once every MMA issued above has completed
-      drain_wait(drain, 0, status);
+      drain_wait(drain, 0, status, kWait);
     }
     __syncthreads();   // (A)
     __syncthreads();   // (B)
@@ -422,11 +432,11 @@ __global__ void __launch_bounds__(Cfg<HS, QB>::kThreads, 1) score_tc_kernel(
       // this warp's queries are consecutive rows of the output
       float* obase = out + ((int64_t)n * geo.T + min(tq0 + q0, geo.T - 1)) * out_stride;
       const int wslot = seg % C::kWBufs;
-      if (ok && !warp_wait(&wfull[wslot], (seg / C::kWBufs) & 1, abort_flag, status)) ok = false;
+      if (ok && !warp_wait(&wfull[wslot], (seg / C::kWBufs) & 1, abort_flag, status, kWait)) ok = false;
       const float* wsm = reinterpret_cast<const float*>(base + C::kWBase + wslot * C::kWBytes);
       for (int j = sg.a; j < sg.b && ok; ++j) {
         const int acc = acc_it % C::kAcc;
-        if (!warp_wait(&accfull[acc], (acc_it / C::kAcc) & 1, abort_flag, status)) {
+        if (!warp_wait(&accfull[acc], (acc_it / C::kAcc) & 1, abort_flag, status, kWait)) {
           ok = false;
           break;
         }
@@ -599,7 +609,7 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
                        const int32_t* pos, const int32_t* tile_off, int units, Units geo,
                        int64_t L, float* out, int64_t out_stride, int* status, uint32_t* hist,
                        const int32_t* gidx, const int32_t* glen, const uint16_t* kraw,
-                       cudaStream_t st) {
+                       const WaitProbe& probe, cudaStream_t st) {
   using C = Cfg<HS, QB>;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB, kGather>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -609,7 +619,7 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return launch_pdl(score_tc_kernel<HS, QB, kGather>, dim3(sms), dim3(C::kThreads),
                     (size_t)C::kSmemBytes, st, tk, tq, wg, pos, tile_off, units, geo, L, out,
-                    out_stride, status, hist, gidx, glen, kraw);
+                    out_stride, status, hist, gidx, glen, kraw, probe);
 }
 
 // Shape of the work units for nh heads and T queries per sequence.
@@ -662,8 +672,12 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
                             int* status, uint32_t* hist, cudaStream_t st, const int32_t* gidx,
-                            const int32_t* glen) {
+                            const int32_t* glen, const WaitProbe* test_probe) {
   const bool gather = gidx != nullptr;
+  WaitProbe probe;
+  probe.wait_cycles = kWaitCycles;
+  probe.skip_tile = -1;
+  if (test_probe) probe = *test_probe;
   const int nh = heads ? hsel : H;
   const Plan p = plan_for(nh, T, gather);
   Units geo;
@@ -690,11 +704,11 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
 #define MISA_TC_CASE(HS_, QB_)                                                                  \
   if (p.HS == HS_ && p.QB == QB_)                                                               \
     return launch_cfg<HS_, QB_, false>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, \
-                                       status, hist, nullptr, nullptr, k, st);
+                                       status, hist, nullptr, nullptr, k, probe, st);
 #define MISA_TC_GATHER_CASE(HS_)                                                                \
   if (p.HS == HS_)                                                                              \
     return launch_cfg<HS_, 1, true>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride,    \
-                                    status, nullptr, gidx, glen, k, st);
+                                    status, nullptr, gidx, glen, k, probe, st);
   if (gather) {
     MISA_TC_GATHER_CASE(16)
     MISA_TC_GATHER_CASE(32)

@@ -756,23 +756,36 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     btop = s_top;
     C = s_total;
   }
-  if (nbulk > 0) {   // bounded wait for the copy; on expiry the row's result is void
+  bool landed = true;
+  if (nbulk > 0) {   // bounded wait for the copy
     long long t0 = clock64();
-    bool landed = true;
     while (!sm100::mbar_try_wait(&lbar, 0)) {
       if (clock64() - t0 > kRowWaitCycles) {
         landed = false;
         break;
       }
     }
-    if (!landed) {   // record it, then give the copy one more bounded wait before going on
+    if (!landed) {   // record it, then give the copy one more bounded wait
       if (t == 0) set_status(status, MISA_ERR_DEVICE_TIMEOUT);
       t0 = clock64();
-      while (!sm100::mbar_try_wait(&lbar, 0) && clock64() - t0 <= kRowWaitCycles) {
+      landed = true;
+      while (!sm100::mbar_try_wait(&lbar, 0)) {
+        if (clock64() - t0 > kRowWaitCycles) {
+          landed = false;
+          break;
+        }
       }
     }
   }
-  __syncthreads();
+  // the threads poll on their own: the row goes on only if every thread saw the copy land;
+  // otherwise its result is void (never read from a row still being written)
+  if (__syncthreads_or(landed ? 0 : 1)) {
+    for (int i = t; i < topk; i += NT) {
+      idx[row * topk + i] = -1;
+      if (vals) vals[row * topk + i] = __int_as_float(0xff800000);
+    }
+    return;
+  }
   // scores -> keys, and in the same pass: the histogram (none given), the bin range (all
   // selected) or this warp's candidate count (cutoff given)
   const uint32_t kgiven = cut << (32 - kScoreHistBits);

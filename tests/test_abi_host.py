@@ -1,4 +1,4 @@
-"""The C-ABI library on the host: it loads, exports every symbol include/misa.h
+"""The C-ABI library on the host: it loads, exports every symbol include/*.h
 declares, sizes workspaces, and rejects invalid arguments before touching the GPU.
 No compute call is made here (CPU only)."""
 
@@ -23,7 +23,8 @@ def lib():
 def test_exports_every_declared_symbol(lib):
     names = lib.declared_symbols()
     assert {"misa_pool_keys", "misa_route_heads", "misa_score_topk", "dsa_score_topk",
-            "misa_dagger_rerank"} <= set(names)
+            "misa_dagger_rerank", "misa_score_topk_noalloc", "misa_testing_score_simt",
+            "misa_testing_score_rows_wait_expiry"} <= set(names)
     cdll = ctypes.CDLL(LIB)
     for n in names:
         assert hasattr(cdll, n), n
@@ -97,9 +98,22 @@ def test_invalid_arguments_rejected_on_host(lib):
     # h > H
     assert c.misa_route_heads(null, null, null, null, null, 1, 1, 8, 128, 1024, 64, 9, null,
                               null, null, 0, null) == 1
-    # h > 16 routed heads is not built
-    assert c.misa_score_topk(null, null, null, null, null, 1, 1, 64, 128, 1024, 17, 16, null,
-                             null, null, null, 0, null) == 2
+    # h > H routed heads; h = 17 .. H is valid (so the null pointers are what is rejected)
+    assert c.misa_score_topk(null, null, null, null, null, 1, 1, 64, 128, 1024, 65, 16, null,
+                             null, null, null, 0, null) == 1
+    assert c.misa_score_topk(null, null, null, null, null, 1, 1, 64, 128, 1024, 64, 16, null,
+                             null, null, null, 0, null) == 1
+    assert c.misa_score_rows(null, null, null, null, null, 1, 1, 64, 128, 1024, 65, null, null,
+                             0, null) == 1
+    assert c.misa_score_topk_noalloc(null, null, null, null, null, 1, 1, 64, 128, 1024, 65, 16,
+                                     null, null, null, null) == 1
+    # test-only entry points: bad wait bound, skip index, gather pair, output stride
+    assert c.misa_testing_score_rows_wait_expiry(null, null, null, null, null, 1, 1, 8, 128, 1024,
+                                                 8, null, null, 0, 10, -1, null) == 1
+    assert c.misa_testing_score_rows_wait_expiry(null, null, null, null, null, 1, 1, 8, 128, 1024,
+                                                 8, null, null, 0, 100000, -2, null) == 1
+    assert c.misa_testing_score_simt(null, null, null, null, null, null, null, 1, 1, 8, 128,
+                                     1024, 8, 512, null, null, 0, null) == 1
     # topk < 1, topk > 16384
     assert c.dsa_score_topk(null, null, null, null, 1, 1, 64, 128, 1024, 0, null, null, null,
                             null, 0, null) == 1
@@ -113,6 +127,6 @@ def test_invalid_arguments_rejected_on_host(lib):
 
 def test_status_strings(lib):
     c = lib.library()
-    for code in range(0, 7):
+    for code in range(0, 8):
         assert c.misa_status_string(code)
     assert c.misa_status_string(99) == b"unknown status"

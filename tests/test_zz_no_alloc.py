@@ -66,6 +66,33 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(M):
                  ref_vals.view(wl.rows, -1), wl.topk)
 
 
+def test_noalloc_matches_oracle_on_every_row_of_the_tiny_workload(M):
+    """The entry point's own scorer and top-k against the fp64 oracle (not only against the
+    workspace entry point): every row of the 16-query, 2K-key workload, with the oracle's
+    routed scores under the heads the GPU routed (Eqs. 9-10)."""
+    import oracle.misa_oracle as orc
+    wl = WORKLOADS["tiny_2k"]
+    x = make_inputs(wl, seed=0)
+    q, w, k, pos = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, wl.B)
+    heads = M.misa_route_heads(q, w, k, kp, pos, wl.B, wl.h)
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    idx, vals = M.misa_score_topk_noalloc(q, w, k, heads, pos, wl.topk, device_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    idx = idx.view(wl.rows, -1).cpu().numpy()
+    vals = vals.view(wl.rows, -1).cpu().numpy()
+    hh = heads.view(wl.rows, -1).cpu().numpy()
+    kk = orc.bf16_bits_to_f64(x.k_bits[0])
+    for t in range(wl.T):
+        P = int(x.pos[0, t]) + 1
+        s_ref = orc.token_scores(orc.bf16_bits_to_f64(x.q_bits[0, t]),
+                                 x.w[0, t].astype(np.float64), kk, P, hh[t])
+        tl.check_selection(idx[t], s_ref, wl.topk, what=f"row {t} set")
+        tl.check_order(idx[t], vals[t], what=f"row {t} order")
+        tl.check_scores(vals[t], s_ref[idx[t]], what=f"row {t} values")
+
+
 def test_noalloc_rejects_calls_beyond_its_scratch(M):
     wl = WORKLOADS["dsv32_decode_32k"].replace(nseq=2, L=4096)
     x = make_inputs(wl, seed=7)

@@ -53,12 +53,11 @@ bool hist_path(int nseq, int T, int64_t L, int nh) {
          !score_tc_block_form(nh, T);
 }
 
-size_t hist_path_bytes(int64_t rows) { return topk_hist_ws_bytes(rows); }
-
-size_t score_ws(int nseq, int T, int64_t L, int nh) {
+size_t score_ws(int nseq, int T, int64_t L, int nh, int topk) {
   const int64_t rows = (int64_t)nseq * T;
   return kStatusBytes + align256((size_t)rows * L * sizeof(float)) +
-         score_tc_ws_bytes(nseq, T, nh) + (hist_path(nseq, T, L, nh) ? hist_path_bytes(rows) : 0);
+         score_tc_ws_bytes(nseq, T, nh) +
+         (hist_path(nseq, T, L, nh) ? topk_hist_ws_bytes(rows, topk) : 0);
 }
 size_t dagger_ws(int nseq, int T, int H, int kprime) {
   const size_t rows = (size_t)nseq * T;
@@ -87,10 +86,10 @@ size_t misa_workspace_size(int op, int nseq, int T, int H, int d, int64_t L, int
       return route_ws(nseq, T, H, L, B);
     case MISA_OP_SCORE_TOPK:
       if (h < 1 || h > H || check_topk(topk) != MISA_OK) return 0;
-      return score_ws(nseq, T, L, h);
+      return score_ws(nseq, T, L, h, topk);
     case MISA_OP_DSA_TOPK:
       if (check_topk(topk) != MISA_OK) return 0;
-      return score_ws(nseq, T, L, H);
+      return score_ws(nseq, T, L, H, topk);
     case MISA_OP_SCORE_ROWS:
       if (h < 1 || h > H) return 0;
       return kStatusBytes + score_tc_ws_bytes(nseq, T, h);
@@ -168,7 +167,7 @@ static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* 
   MISA_TRY(check_opt(vals, rows * topk * 4, 4));
   MISA_TRY(check_opt(scores, rows * L * 4, 4));
   const int nh = heads ? h : H;
-  MISA_TRY(check_ws(ws, ws_bytes, score_ws(nseq, T, L, nh)));
+  MISA_TRY(check_ws(ws, ws_bytes, score_ws(nseq, T, L, nh, topk)));
   cudaStream_t st = (cudaStream_t)stream;
   float* sc = scores ? scores : reinterpret_cast<float*>(ws_region(ws, 0));
   int* status = status_word(ws);

@@ -144,8 +144,9 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
 cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
                              const uint32_t* hist, uint64_t* cand, uint32_t* gcount, int rows,
                              int topk, int32_t* idx, float* vals, int* status, cudaStream_t st);
-// Scratch of the histogram path: histogram, group counts, group buffers (256-aligned each).
-size_t topk_hist_ws_bytes(int64_t rows);
+// Scratch of the histogram path: histogram, group counts, group buffers (ceil(topk / 1024)
+// groups of 8192 pairs per row), each region 256-aligned.
+size_t topk_hist_ws_bytes(int64_t rows, int topk);
 
 // Power-of-two length of the shared-memory sort buffer for `topk` entries (topk.cu).
 int topk_sort_size(int topk);

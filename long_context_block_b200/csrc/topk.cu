@@ -362,9 +362,16 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(
 // one group) are done by topk_hist_overflow_kernel with an exact radix select.
 constexpr int kSelThreads = 256;
 constexpr int kGroupSpan = 1024;                          // output positions per group
-constexpr int kMaxGroups = kTopkCandCap / kGroupSpan;     // 16 CTAs per row
-constexpr int kGroupBuf = 4096;                           // pairs one group CTA holds
+constexpr int kMaxGroups = kTopkCandCap / kGroupSpan;     // at most 16 CTAs per row
+constexpr int kGroupBuf = 8192;                           // pairs one group CTA holds
 constexpr uint32_t kBigBin = kGroupBuf - kGroupSpan;      // larger bins: overflow path
+constexpr int kGroupExactMax = 4096;   // overflow rows up to this k: CTA 0 of the group kernel
+
+// Groups of a row: a bin at or above the cutoff starts before output position k, so its
+// group is below ceil(k / kGroupSpan).
+__host__ __device__ constexpr int hist_groups(int topk) {
+  return (topk + kGroupSpan - 1) / kGroupSpan;
+}
 constexpr int kScatterPer = 16;                           // scores per thread in pass 1
 constexpr int kScatterChunk = kSelThreads * kScatterPer;  // 4096 scores per CTA
 
@@ -488,7 +495,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_scatter_kernel(
   __syncthreads();
   if (t < kMaxGroups && lcount[t]) lbase[t] = atomicAdd(&gcount[row * kMaxGroups + t], lcount[t]);
   __syncthreads();
-  uint64_t* crow = cand + row * (int64_t)(kMaxGroups * kGroupBuf);
+  uint64_t* crow = cand + row * (int64_t)hist_groups(topk) * kGroupBuf;
 #pragma unroll
   for (int j = 0; j < kScatterPer; ++j) {
     if (slot[j] == 0xffffffffu) continue;
@@ -500,7 +507,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_scatter_kernel(
 }
 
 // Pass 2: CTA g of a row sorts group g's candidates and writes them at their positions.
-__global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
+__global__ void __launch_bounds__(kSelThreads, 1) topk_group_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
     const uint32_t* __restrict__ hist, int topk, const uint64_t* __restrict__ cand,
     int32_t* __restrict__ idx, float* __restrict__ vals) {
@@ -524,7 +531,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
   if (hist_overflow(s_total, s_big)) {
     // crowded cutoff (e.g. many equal scores): an exact selection over the whole row, here
     // by CTA 0 when the selected pairs fit its buffer, else by topk_hist_overflow_kernel
-    if (g != 0 || topk > kGroupBuf) return;
+    if (g != 0 || topk > kGroupExactMax) return;
     int sortn = kSelThreads;
     while (sortn < topk) sortn <<= 1;
     select_row_global_nt<kSelThreads>(scores + row * stride, nullptr, n, topk, sortn, gbuf, buckets,
@@ -578,7 +585,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
   const uint32_t cnt = min(s_cnt, (uint32_t)kGroupBuf);
   if (cnt == 0) return;
   const uint32_t blo = s_lo, bhi = s_hi, start = s_start;
-  const uint64_t* src = cand + row * (int64_t)(kMaxGroups * kGroupBuf) + g * kGroupBuf;
+  const uint64_t* src = cand + row * (int64_t)hist_groups(topk) * kGroupBuf + g * kGroupBuf;
   for (uint32_t i = t; i < cnt; i += kSelThreads) gathered[i] = src[i];
   __syncthreads();
   if (!group_sort_desc<kSelThreads>(gathered, cnt, sorted, buckets, blo, bhi, warp_sums, s_flag)) {
@@ -587,12 +594,13 @@ __global__ void __launch_bounds__(kSelThreads, 2) topk_group_kernel(
     while ((uint32_t)sortn < cnt) sortn <<= 1;
     for (int i = t; i < sortn; i += kSelThreads) sorted[i] = (uint32_t)i < cnt ? gathered[i] : 0ull;
     __syncthreads();
-    switch (sortn / kSelThreads) {   // cnt <= kGroupBuf = 16 * kSelThreads
+    switch (sortn / kSelThreads) {   // cnt <= kGroupBuf = 32 * kSelThreads
       case 1: sort_buf_desc_e<1, kSelThreads>(sorted); break;
       case 2: sort_buf_desc_e<2, kSelThreads>(sorted); break;
       case 4: sort_buf_desc_e<4, kSelThreads>(sorted); break;
       case 8: sort_buf_desc_e<8, kSelThreads>(sorted); break;
-      default: sort_buf_desc_e<16, kSelThreads>(sorted); break;
+      case 16: sort_buf_desc_e<16, kSelThreads>(sorted); break;
+      default: sort_buf_desc_e<32, kSelThreads>(sorted); break;
     }
   }
   for (uint32_t i = t; i < cnt && start + i < target; i += kSelThreads) {
@@ -1038,9 +1046,9 @@ cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t*
   e = cudaFuncSetAttribute(topk_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(topk_group_kernel, dim3(kMaxGroups, (unsigned)rows), dim3(kSelThreads), smem, st,
+  e = launch_pdl(topk_group_kernel, dim3(hist_groups(topk), (unsigned)rows), dim3(kSelThreads), smem, st,
                  scores, stride, pos, L, hist, topk, (const uint64_t*)cand, idx, vals);
-  if (e != cudaSuccess || topk <= kGroupBuf) return e;   // the group kernel covers overflow rows
+  if (e != cudaSuccess || topk <= kGroupExactMax) return e;   // the group kernel covers overflow rows
   const int sortn = topk_sort_size(topk);
   const size_t ov_smem = (size_t)sortn * sizeof(uint64_t);
   e = cudaFuncSetAttribute(topk_hist_overflow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1050,9 +1058,9 @@ cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t*
                     stride, pos, L, hist, topk, sortn, idx, vals);
 }
 
-size_t topk_hist_ws_bytes(int64_t rows) {
+size_t topk_hist_ws_bytes(int64_t rows, int topk) {
   return align256((size_t)rows * kScoreHistBins * 4) + align256((size_t)rows * kMaxGroups * 4) +
-         align256((size_t)rows * kMaxGroups * kGroupBuf * 8);
+         align256((size_t)rows * hist_groups(topk) * kGroupBuf * 8);
 }
 
 // Cluster size for rows of up to `len` scores, or 0 when the cluster form does not fit.

@@ -42,10 +42,13 @@ def test_workspace_sizes(lib):
     a256 = lambda x: (x + 255) // 256 * 256
     tc = lambda rows, n: a256(rows * n * 256) + a256(rows * n * 4) + a256((rows + 1) * 4)
     # rows of 8192+ scores (at most 1024 rows) add the histogram top-k scratch: per row a
-    # 4096-bin score histogram, 16 group counts and 16 group buffers of 4096 pairs
-    hp = lambda rows: a256(rows * 4096 * 4) + a256(rows * 16 * 4) + a256(rows * 16 * 4096 * 8)
-    assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 16) + hp(32)
-    assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 64) + hp(32)
+    # 4096-bin score histogram, 16 group counts and ceil(k / 1024) group buffers of 8192 pairs
+    hp = lambda rows, k: (a256(rows * 4096 * 4) + a256(rows * 16 * 4)
+                          + a256(rows * (-(-k // 1024)) * 8192 * 8))
+    assert ws(2, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 16) + hp(32, 2048)
+    assert ws(3, 32, 1, 64, 128, 32768, 64, 8, 2048, 8192) == 256 + 32 * 32768 * 4 + tc(32, 64) + hp(32, 2048)
+    assert ws(2, 16, 1, 64, 128, 131072, 64, 8, 8192, 8192) == \
+        256 + 16 * 131072 * 4 + tc(16, 16) + hp(16, 8192)
     # 16 queries of one sequence share key tiles: one unit of 16 queries x 8 slots
     assert ws(2, 1, 16, 64, 128, 2048, 64, 8, 256, 512) == 256 + 16 * 2048 * 4 + tc(1, 128)
     # re-rank: sorted candidate ids, their scores, per-row counts, tensor-core scratch

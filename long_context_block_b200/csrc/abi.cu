@@ -37,7 +37,8 @@ int check_topk(int topk) {
 }
 
 size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
-  if (route_tc_supported(nseq, T, H, L, B)) return kStatusBytes + route_tc_ws_bytes(nseq, T, H);
+  if (route_tc_supported(nseq, T, H, L, B))
+    return kStatusBytes + route_tc_ws_bytes(nseq, T, H, L, B);
   const int64_t M = (L + B - 1) / B;
   const int64_t nchunk = (M + kRouteChunk - 1) / kRouteChunk;
   return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float)) +

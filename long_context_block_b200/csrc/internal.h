@@ -78,10 +78,11 @@ cudaError_t launch_hisa(const uint16_t* q, const float* w, const uint16_t* k, co
                         int* status, cudaStream_t st);
 
 // K2 -- router on tcgen05 for sequences with many queries (route_tc.cu): the full-block
-// part of Eq. (7) as a GEMM against the sequence's pooled keys (bf16 hi + lo), the partial
-// block on CUDA cores, then the top-h.  needs route_tc_ws_bytes(...) of scratch.
+// part of Eq. (7) as a GEMM against the sequence's pooled keys (bf16 hi + lo, chunks of 256
+// blocks), the partial block on CUDA cores, then the top-h.  needs route_tc_ws_bytes(...)
+// of scratch.
 bool route_tc_supported(int nseq, int T, int H, int64_t L, int B);
-size_t route_tc_ws_bytes(int nseq, int T, int H);
+size_t route_tc_ws_bytes(int nseq, int T, int H, int64_t L, int B);
 cudaError_t launch_route_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const float* k_pool, const int32_t* pos, int nseq, int T, int H,
                             int64_t L, int B, int h, int32_t* heads, float* E, void* scratch,

@@ -2,17 +2,26 @@
 // (Methodology section 1), for sequences with many queries (prefill):
 //
 //   E[t,j] = |w[t,j]| / M_t * ( sum_{b < Mfull_t} ReLU(q[t,j] . kp_b) + ReLU(q[t,j] . kpart_t) )
+//   heads_t = the h largest E[t,j]  (ties: lower j)
 //
 // where Mfull_t = floor(P_t / B) full blocks come from the pooled keys and kpart_t, the
 // mean of the keys of query t's partial last block (present when P_t mod B != 0), is
 // added on CUDA cores.  The full-block part is a GEMM: A = the (query, head) rows of q
 // (128 rows = 128 / H queries per tile, streamed by TMA), B = the sequence's pooled keys
-// (up to 256 blocks, resident in shared memory).  Pooled keys are fp32; they are split
-// into bf16 hi + lo (hi = bf16(kp), lo = bf16(kp - hi)) so that two bf16 MMAs reproduce
-// the fp32 products to about 2^-16 relative.  Accumulators live in TMEM (N = the tile's
-// largest full-block count, rounded up to 16); the epilogue masks each row's columns to
-// its own causal block count, adds the partial block and writes E.  The top-h selection
-// runs afterwards, one warp per query.
+// in chunks of 256 blocks (one chunk resident in shared memory at a time).  A tile makes
+// one MMA item per chunk its queries reach (even tiles walk their chunks upward, odd tiles
+// downward, so consecutive items mostly share the resident chunk).  Pooled keys are fp32;
+// they are split into bf16 hi + lo (hi = bf16(kp), lo = bf16(kp - hi)) so that two bf16
+// MMAs reproduce the fp32 products to about 2^-16 relative.  Accumulators live in TMEM
+// (N = the item's largest full-block count within its chunk, rounded up to 16).
+//
+// Epilogue: 8 warps, two per TMEM lane quarter; the two warps of a quarter split the
+// accumulator columns (masked to each row's own causal block count) and the partial-block
+// dot product (64 dimensions each), which reads the query rows from the tile's A stage
+// (the stage is released by the epilogue, not by the MMA) and the tile's partial pooled
+// keys from a shared-memory copy loaded with the A tile.  The halves are combined through
+// shared memory, E is written (when asked for), and every row ranks its head among its
+// query's H energies to write the top-h heads.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -29,22 +38,30 @@ using namespace sm100;
 constexpr int kRows = 128;                          // (query, head) rows per tile
 constexpr int kATileBytes = kRows * kHeadDim * 2;   // 32 KB
 constexpr int kAHalf = kATileBytes / 2;
-constexpr int kMaxBlocks = 256;                     // pooled keys held for one sequence
+constexpr int kMaxBlocks = 256;                     // pooled keys per chunk (one resident)
 constexpr int kBBytes = kMaxBlocks * kHeadDim * 2;  // 64 KB per part (hi or lo)
 constexpr int kBHalf = kBBytes / 2;
+constexpr int kMaxQT = 16;                          // queries per tile (H >= 8)
+constexpr int kKpBytes = kMaxQT * kHeadDim * 4;     // partial pooled keys of a tile (fp32)
 constexpr int kStages = 2;
 constexpr int kAcc = 2;
 constexpr int kCols = 512;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr long long kWaitCycles = 4000000000LL;
 
 constexpr int kStageBase = 0;
 constexpr int kBBase = kStages * kATileBytes;         // hi then lo
-constexpr int kBarBase = kBBase + 2 * kBBytes;
+constexpr int kKpBase = kBBase + 2 * kBBytes;
+constexpr int kEsBase = kKpBase + kStages * kKpBytes;  // E of the tile's rows
+constexpr int kXBase = kEsBase + kRows * 4;            // second half's sums: [2][kRows]
+constexpr int kBarBase = kXBase + 2 * kRows * 4;
 // full[S], empty[S], bfull, bempty, accfull[A], accempty[A], drain
 constexpr int kNumBars = 2 * kStages + 2 + 2 * kAcc + 1;
 constexpr int kMiscBase = kBarBase + kNumBars * 8;
 constexpr int kSmemBytes = kMiscBase + 16 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
   volatile int never = 0;
@@ -58,27 +75,35 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+}
+
 struct RouteGeo {
   int T, H, B, QT;   // queries per sequence, heads, block size, queries per tile
   int64_t L;
   int tiles_per_seq;
+  int mpad;          // pooled-key rows per sequence in the hi / lo copies (chunks of 256)
 };
 
-// Largest full-block count among the queries of tile i (0 .. 256).
+// Largest full-block count among the queries of tile i.
 __device__ __forceinline__ int tile_blocks(const int32_t* pos, const RouteGeo& g, int i) {
   const int n = i / g.tiles_per_seq;
   const int ta = (i % g.tiles_per_seq) * g.QT;
   int mf = 0;
   for (int qq = 0; qq < g.QT && ta + qq < g.T; ++qq)
     mf = max(mf, prefix_len(pos, (int64_t)n * g.T + ta + qq, g.L, nullptr) / g.B);
-  return min(mf, kMaxBlocks);
+  return mf;
 }
+// MMA items of a tile whose queries reach mf full blocks, and the chunk of its k-th item.
+__device__ __forceinline__ int tile_items(int mf) { return max(1, (mf + kMaxBlocks - 1) / kMaxBlocks); }
+__device__ __forceinline__ int item_chunk(int i, int k, int nc) { return (i & 1) ? nc - 1 - k : k; }
 
 __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
-    const __grid_constant__ CUtensorMap tm_lo, const uint16_t* __restrict__ q,
-    const float* __restrict__ w, const float* __restrict__ kpart, const int32_t* __restrict__ pos,
-    RouteGeo g, int total_tiles, float* __restrict__ E, int* status) {
+    const __grid_constant__ CUtensorMap tm_lo, const float* __restrict__ w,
+    const float* __restrict__ kpart, const int32_t* __restrict__ pos, RouteGeo g, int total_tiles,
+    int h, int32_t* __restrict__ heads, float* __restrict__ E, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = (int)((int64_t)total_tiles * blockIdx.x / gridDim.x);
@@ -96,10 +121,16 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kMiscBase);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kMiscBase + 4);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + kEpiWarps);   // the MMAs' commit and every epilogue warp
+    }
     mbar_init(bfull, 1);
     mbar_init(bempty, 1);
-    for (int a = 0; a < kAcc; ++a) { mbar_init(&accfull[a], 1); mbar_init(&accempty[a], 128); }
+    for (int a = 0; a < kAcc; ++a) {
+      mbar_init(&accfull[a], 1);
+      mbar_init(&accempty[a], kEpiThreads);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -109,34 +140,47 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const uint32_t kp_bytes = (uint32_t)g.QT * kHeadDim * 4;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     int issued = 0, bissued = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
-      int cur_seq = -1;
-      for (int i = t0; i < t1; ++i) {
+      int64_t cur_key = -1;   // resident chunk: sequence * 65536 + chunk
+      bool ok = true;
+      for (int i = t0; i < t1 && ok; ++i) {
         const int n = i / g.tiles_per_seq;
-        if (n != cur_seq) {   // pooled keys of a new sequence (after the last MMAs on the old)
-          if (!mbar_wait(bempty, (bissued & 1) ^ 1, abort_flag, status, kWaitCycles)) break;
-          mbar_arrive_expect_tx(bfull, 2 * kBBytes);
-          uint8_t* hb = base + kBBase;
-          tma_load_2d(hb, &tm_hi, bfull, 0, n * kMaxBlocks);
-          tma_load_2d(hb + kBHalf, &tm_hi, bfull, 64, n * kMaxBlocks);
-          tma_load_2d(hb + kBBytes, &tm_lo, bfull, 0, n * kMaxBlocks);
-          tma_load_2d(hb + kBBytes + kBHalf, &tm_lo, bfull, 64, n * kMaxBlocks);
-          ++bissued;
-          cur_seq = n;
-        }
         const int s = issued % kStages;
         if (!mbar_wait(&empty[s], ((issued / kStages) & 1) ^ 1, abort_flag, status, kWaitCycles))
           break;
         uint8_t* ab = base + kStageBase + s * kATileBytes;
-        mbar_arrive_expect_tx(&full[s], kATileBytes);
+        const int64_t qrow0 = (int64_t)n * g.T + (int64_t)(i % g.tiles_per_seq) * g.QT;
+        mbar_arrive_expect_tx(&full[s], kATileBytes + kp_bytes);
         tma_load_2d(ab, &tm_q, &full[s], 0, i * kRows);
         tma_load_2d(ab + kAHalf, &tm_q, &full[s], 64, i * kRows);
+        bulk_load(base + kKpBase + s * kKpBytes, kpart + qrow0 * kHeadDim, kp_bytes, &full[s]);
         ++issued;
+        const int nc = tile_items(tile_blocks(pos, g, i));
+        for (int k = 0; k < nc; ++k) {
+          const int c = item_chunk(i, k, nc);
+          const int64_t key = (int64_t)n * 65536 + c;
+          if (key == cur_key) continue;
+          // a new chunk of pooled keys, after the last MMAs on the resident one
+          if (!mbar_wait(bempty, (bissued & 1) ^ 1, abort_flag, status, kWaitCycles)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bfull, 2 * kBBytes);
+          uint8_t* hb = base + kBBase;
+          const int row = n * g.mpad + c * kMaxBlocks;
+          tma_load_2d(hb, &tm_hi, bfull, 0, row);
+          tma_load_2d(hb + kBHalf, &tm_hi, bfull, 64, row);
+          tma_load_2d(hb + kBBytes, &tm_lo, bfull, 0, row);
+          tma_load_2d(hb + kBBytes + kBHalf, &tm_lo, bfull, 64, row);
+          ++bissued;
+          cur_key = key;
+        }
       }
     }
     __syncthreads();   // (A)
@@ -150,44 +194,57 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t smem0 = smem_u32(base);
-      int it = 0, bseen = 0, cur_seq = -1;
+      int it = 0, acc_it = 0, bseen = 0;
+      int64_t cur_key = -1;
       bool ok = true;
       for (int i = t0; i < t1 && ok; ++i) {
         const int n = i / g.tiles_per_seq;
-        if (n != cur_seq) {
-          if (cur_seq >= 0) mma_commit(bempty);   // the old pooled keys may be replaced
-          if (!mbar_wait(bfull, bseen & 1, abort_flag, status, kWaitCycles)) break;
-          ++bseen;
-          cur_seq = n;
-        }
         const int s = it % kStages;
-        const int acc = it % kAcc;
-        if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, status, kWaitCycles) ||
-            !mbar_wait(&accempty[acc], ((it / kAcc) & 1) ^ 1, abort_flag, status, kWaitCycles)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int nb = tile_blocks(pos, g, i);
-        const int N = (nb + 15) & ~15;
-        if (N > 0) {
-          const uint32_t idesc = idesc_bf16_f32(128, N);
-          const uint32_t aaddr = smem0 + kStageBase + s * kATileBytes;
-          const uint32_t d = tmem_base + (uint32_t)(acc * 256);
+        if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, status, kWaitCycles)) break;
+        const int mf = tile_blocks(pos, g, i);
+        const int nc = tile_items(mf);
+        for (int k = 0; k < nc && ok; ++k) {
+          const int c = item_chunk(i, k, nc);
+          const int64_t key = (int64_t)n * 65536 + c;
+          if (key != cur_key) {
+            if (cur_key >= 0) mma_commit(bempty);   // the resident chunk may be replaced
+            if (!mbar_wait(bfull, bseen & 1, abort_flag, status, kWaitCycles)) {
+              ok = false;
+              break;
+            }
+            ++bseen;
+            cur_key = key;
+          }
+          const int acc = acc_it % kAcc;
+          if (!mbar_wait(&accempty[acc], ((acc_it / kAcc) & 1) ^ 1, abort_flag, status,
+                         kWaitCycles)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nb = min(max(mf - c * kMaxBlocks, 0), kMaxBlocks);
+          const int N = (nb + 15) & ~15;
+          if (N > 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, N);
+            const uint32_t aaddr = smem0 + kStageBase + s * kATileBytes;
+            const uint32_t d = tmem_base + (uint32_t)(acc * 256);
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const uint32_t baddr = smem0 + kBBase + part * kBBytes;
+            for (int part = 0; part < 2; ++part) {
+              const uint32_t baddr = smem0 + kBBase + part * kBBytes;
 #pragma unroll
-            for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-              const uint32_t ao = (kk >> 2) * kAHalf + (kk & 3) * 32;
-              const uint32_t bo = (kk >> 2) * kBHalf + (kk & 3) * 32;
-              mma_bf16(d, desc_kmajor_sw128(aaddr + ao), desc_kmajor_sw128(baddr + bo), idesc,
-                       (part | kk) ? 1u : 0u);
+              for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * kAHalf + (kk & 3) * 32;
+                const uint32_t bo = (kk >> 2) * kBHalf + (kk & 3) * 32;
+                mma_bf16(d, desc_kmajor_sw128(aaddr + ao), desc_kmajor_sw128(baddr + bo), idesc,
+                         (part | kk) ? 1u : 0u);
+              }
             }
           }
+          mma_commit(&accfull[acc]);
+          ++acc_it;
         }
-        mma_commit(&empty[s]);
-        mma_commit(&accfull[acc]);
+        if (!ok) break;
+        mma_commit(&empty[s]);   // the tile's A stage, once all its items' MMAs are done
         ++it;
       }
       mma_commit(drain);
@@ -198,58 +255,109 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     tc_fence_after();
     tmem_dealloc(tmem_base, kCols);
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-5)
-    const int quarter = warp & 3;
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    const int e = warp - 2;
+    const int grp = e >> 2;              // 0: even column chunks, dims 0-63; 1: odd, 64-127
+    const int quarter = warp & 3;        // TMEM lanes this warp may read
     const int r = quarter * 32 + lane;   // row of the tile
+    const int qq = r / g.H, j = r % g.H;
+    float* Es = reinterpret_cast<float*>(base + kEsBase);
+    float* xsum = reinterpret_cast<float*>(base + kXBase);
+    float* xdot = xsum + kRows;
+    // Every epilogue warp walks every tile and meets both named barriers of each, whatever
+    // happens; after a failed (bounded) wait a warp only skips the work.
     bool ok = true;
-    int it = 0;
-    for (int i = t0; i < t1 && ok; ++i, ++it) {
-      const int acc = it % kAcc;
-      if (!warp_wait(&accfull[acc], (it / kAcc) & 1, abort_flag, status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    int it = 0, acc_it = 0;
+    for (int i = t0; i < t1; ++i, ++it) {
+      const int s = it % kStages;
       const int n = i / g.tiles_per_seq;
-      const int tq = (i % g.tiles_per_seq) * g.QT + r / g.H;   // query index in the sequence
-      const int j = r % g.H;
+      const int ta = (i % g.tiles_per_seq) * g.QT;
+      const int tq = ta + qq;
       const bool valid = tq < g.T;
       const int64_t qrow = (int64_t)n * g.T + (valid ? tq : 0);
       const int P = prefix_len(pos, qrow, g.L, nullptr);
-      const int mfull = min(P / g.B, kMaxBlocks);
-      // warp-uniform column count (queries of a warp may differ when H < 32)
-      int mwarp = mfull;
+      const int mfull = P / g.B;
+      const int M = (P + g.B - 1) / g.B;
+      const float wabs = fabsf(w[qrow * g.H + j]);
+      const int nc = tile_items(tile_blocks(pos, g, i));
+      float sum = 0.f, dot = 0.f;
+      // the partial last block first: its half of q . kpart (64 dimensions) reads the query
+      // row from the tile's A stage and the partial keys copied with it, as soon as they
+      // landed, and then releases the stage
+      if (ok && !warp_wait(&full[s], (it / kStages) & 1, abort_flag, status)) ok = false;
+      if (ok && M > mfull) {
+        const uint8_t* arow = base + kStageBase + s * kATileBytes + grp * kAHalf + r * 128;
+        const float4* kv = reinterpret_cast<const float4*>(base + kKpBase + s * kKpBytes +
+                                                           (qq * kHeadDim + grp * 64) * 4);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mwarp = max(mwarp, __shfl_xor_sync(0xffffffffu, mwarp, o));
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
-      float sum = 0.f;
-      for (int c0 = 0; c0 < mwarp; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + c0, v);
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if (c0 + c < mfull) sum += fmaxf(v[c], 0.f);
-      }
-      tc_fence_before();
-      mbar_arrive(&accempty[acc]);
-      if (valid) {
-        const int M = (P + g.B - 1) / g.B;
-        if (M > mfull) {   // the partial last block of this prefix
-          const uint4* qv = reinterpret_cast<const uint4*>(q + (qrow * g.H + j) * kHeadDim);
-          const float4* kv = reinterpret_cast<const float4*>(kpart + qrow * kHeadDim);
-          float dt = 0.f;
-#pragma unroll 4
-          for (int c = 0; c < kHeadDim / 8; ++c) {
-            const uint4 x = qv[c];
-            const float4 a = kv[2 * c], b = kv[2 * c + 1];
-            dt = fmaf(bf16lo(x.x), a.x, dt); dt = fmaf(bf16hi(x.x), a.y, dt);
-            dt = fmaf(bf16lo(x.y), a.z, dt); dt = fmaf(bf16hi(x.y), a.w, dt);
-            dt = fmaf(bf16lo(x.z), b.x, dt); dt = fmaf(bf16hi(x.z), b.y, dt);
-            dt = fmaf(bf16lo(x.w), b.z, dt); dt = fmaf(bf16hi(x.w), b.w, dt);
-          }
-          sum += fmaxf(dt, 0.f);
+        for (int c = 0; c < 8; ++c) {   // 16-byte chunk c of the row (128-byte swizzle)
+          const uint4 x = *reinterpret_cast<const uint4*>(arow + ((c ^ (r & 7)) << 4));
+          const float4 a = kv[2 * c], b = kv[2 * c + 1];
+          dot = fmaf(bf16lo(x.x), a.x, dot); dot = fmaf(bf16hi(x.x), a.y, dot);
+          dot = fmaf(bf16lo(x.y), a.z, dot); dot = fmaf(bf16hi(x.y), a.w, dot);
+          dot = fmaf(bf16lo(x.z), b.x, dot); dot = fmaf(bf16hi(x.z), b.y, dot);
+          dot = fmaf(bf16lo(x.w), b.z, dot); dot = fmaf(bf16hi(x.w), b.w, dot);
         }
-        E[qrow * g.H + j] = fabsf(w[qrow * g.H + j]) * sum / (float)M;
+      }
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&empty[s]);   // this warp is done with the stage
+      for (int k = 0; k < nc; ++k, ++acc_it) {   // the tile's items, one chunk each
+        const int acc = acc_it % kAcc;
+        // this row's full blocks inside the item's chunk, and the warp's largest count
+        const int mrow = min(max(mfull - item_chunk(i, k, nc) * kMaxBlocks, 0), kMaxBlocks);
+        int mwarp = mrow;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+          mwarp = max(mwarp, __shfl_xor_sync(0xffffffffu, mwarp, o));
+        if (ok && !warp_wait(&accfull[acc], (acc_it / kAcc) & 1, abort_flag, status)) ok = false;
+        if (ok) {
+          tc_fence_after();
+          const uint32_t taddr =
+              tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
+          for (int c0 = 16 * grp; c0 < mwarp; c0 += 32) {
+            float v[16];
+            tmem_ld16(taddr + c0, v);
+            if (c0 + 16 <= mrow) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) sum += fmaxf(v[c], 0.f);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                if (c0 + c < mrow) sum += fmaxf(v[c], 0.f);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&accempty[acc]);
+        }
+      }
+      if (grp == 1) {
+        xsum[r] = sum;
+        xdot[r] = dot;
+      }
+      epi_bar();
+      if (grp == 0) {
+        const float tot = sum + xsum[r] + (M > mfull ? fmaxf(dot + xdot[r], 0.f) : 0.f);
+        const float ev = wabs * tot / (float)M;
+        Es[r] = ev;
+        if (ok && valid && E) E[qrow * g.H + j] = ev;
+      }
+      epi_bar();
+      // top-h heads: each row (one head of one query) counts the heads of its query that
+      // come before it (larger E, or equal E and a lower index) and writes its own index at
+      // that rank when the rank is below h
+      if (grp == 0 && ok && valid) {   // H is a multiple of 8: four energies per load
+        const float ev = Es[r];
+        const float4* eq = reinterpret_cast<const float4*>(Es + qq * g.H);
+        int rank = 0;
+        for (int j4 = 0; j4 < g.H / 4; ++j4) {
+          const float4 o = eq[j4];
+          const int jb = 4 * j4;
+          rank += (o.x > ev || (o.x == ev && jb < j)) ? 1 : 0;
+          rank += (o.y > ev || (o.y == ev && jb + 1 < j)) ? 1 : 0;
+          rank += (o.z > ev || (o.z == ev && jb + 2 < j)) ? 1 : 0;
+          rank += (o.w > ev || (o.w == ev && jb + 3 < j)) ? 1 : 0;
+        }
+        if (rank < h) heads[qrow * h + rank] = j;
       }
     }
     __syncthreads();   // (A)
@@ -257,72 +365,50 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
   }
 }
 
-// Pooled keys fp32 -> bf16 hi + lo, [nseq, 256, 128] each, zero rows past the sequence's
-// blocks; grid = nseq * 256 blocks of 128 threads.
-__global__ void route_tc_split_kernel(const float* __restrict__ k_pool, int Mpool,
+// Pooled keys fp32 -> bf16 hi + lo, [nseq, mpad, 128] each (mpad = Mpool rounded up to
+// whole chunks), zero rows past the sequence's blocks; grid = nseq * mpad blocks of 128
+// threads.
+__global__ void route_tc_split_kernel(const float* __restrict__ k_pool, int Mpool, int mpad,
                                       uint16_t* __restrict__ hi, uint16_t* __restrict__ lo) {
-  const int n = blockIdx.x / kMaxBlocks, b = blockIdx.x % kMaxBlocks, d = threadIdx.x;
+  const int n = blockIdx.x / mpad, b = blockIdx.x % mpad, d = threadIdx.x;
   const float x = b < Mpool ? k_pool[((int64_t)n * Mpool + b) * kHeadDim + d] : 0.f;
-  const __nv_bfloat16 h = __float2bfloat16_rn(x);
-  const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
-  const int64_t o = ((int64_t)n * kMaxBlocks + b) * kHeadDim + d;
-  hi[o] = __bfloat16_as_ushort(h);
+  const __nv_bfloat16 hh = __float2bfloat16_rn(x);
+  const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(hh));
+  const int64_t o = ((int64_t)n * mpad + b) * kHeadDim + d;
+  hi[o] = __bfloat16_as_ushort(hh);
   lo[o] = __bfloat16_as_ushort(l);
 }
 
-// Mean of each query's partial last block (keys Mfull*B .. P-1); grid = rows, 128 threads.
-__global__ void route_tc_partial_kernel(const uint16_t* __restrict__ k, const int32_t* __restrict__ pos,
-                                        int T, int64_t L, int B, float* __restrict__ kpart,
-                                        int* status) {
-  const int64_t row = blockIdx.x;
-  const int d = threadIdx.x;
-  const int P = prefix_len(pos, row, L, d == 0 ? status : nullptr);
-  const int s0 = (P / B) * B, cnt = P - s0;
-  float a = 0.f;
-  if (cnt > 0) {
-    const uint16_t* kr = k + ((row / T) * L + s0) * kHeadDim + d;
-    for (int s = 0; s < cnt; ++s) a += bf16_to_f32(kr[(int64_t)s * kHeadDim]);
-    a /= (float)cnt;
-  }
-  kpart[row * kHeadDim + d] = a;
-}
-
-__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
-}
-
-// Top-h of E per query (one warp per query): descending E, ties to the lower head.
-__global__ void route_tc_select_kernel(const float* __restrict__ E, int rows, int H, int h,
-                                       int32_t* __restrict__ heads) {
+// Mean of each query's partial last block (keys Mfull*B .. P-1), zero when there is none:
+// one warp per query, lane l sums dimensions 4l .. 4l+3 (the warp reads whole key rows).
+constexpr int kPartWarps = 8;
+__global__ void __launch_bounds__(32 * kPartWarps) route_tc_partial_kernel(
+    const uint16_t* __restrict__ k, const int32_t* __restrict__ pos, int rows, int T, int64_t L,
+    int B, float* __restrict__ kpart, int* status) {
+  const int64_t row = (int64_t)blockIdx.x * kPartWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (row >= rows) return;
-  constexpr int kPer = MISA_MAX_HEADS / 32;
-  float e[kPer];
+  const int P = prefix_len(pos, row, L, lane == 0 ? status : nullptr);
+  const int s0 = (P / B) * B, cnt = P - s0;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  const uint2* kr = reinterpret_cast<const uint2*>(k + ((row / T) * L + s0) * kHeadDim) + lane;
+  int s = 0;
+  for (; s + 4 <= cnt; s += 4) {
+    uint2 v[4];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = lane + 32 * i;
-    e[i] = j < H ? E[row * H + j] : -1.f;
-  }
-  for (int r = 0; r < h; ++r) {
-    float bv = -1.f;
-    int bi = 0x7fffffff;
+    for (int u = 0; u < 4; ++u) v[u] = kr[(int64_t)(s + u) * (kHeadDim / 4)];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int j = lane + 32 * i;
-      if (e[i] >= 0.f && better(e[i], j, bv, bi)) { bv = e[i]; bi = j; }
+    for (int u = 0; u < 4; ++u) {
+      a0 += bf16lo(v[u].x); a1 += bf16hi(v[u].x); a2 += bf16lo(v[u].y); a3 += bf16hi(v[u].y);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-    }
-    if (lane == 0) heads[row * h + r] = bi;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (lane + 32 * i == bi) e[i] = -1.f;
   }
+  for (; s < cnt; ++s) {
+    const uint2 v = kr[(int64_t)s * (kHeadDim / 4)];
+    a0 += bf16lo(v.x); a1 += bf16hi(v.x); a2 += bf16lo(v.y); a3 += bf16hi(v.y);
+  }
+  const float inv = cnt > 0 ? 1.f / (float)cnt : 0.f;
+  reinterpret_cast<float4*>(kpart + row * kHeadDim)[lane] =
+      make_float4(a0 * inv, a1 * inv, a2 * inv, a3 * inv);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -359,19 +445,27 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t nrows, uint32_t box_rows
 
 }  // namespace
 
-bool route_tc_supported(int nseq, int T, int H, int64_t L, int B) {
-  if (H < 1 || H > 128 || (128 % H) != 0 || encode_fn() == nullptr) return false;
-  const int QT = 128 / H;
+// Rows per sequence of the hi / lo pooled-key copies: whole chunks of kMaxBlocks.
+static int64_t route_tc_mpad(int64_t L, int B) {
   const int64_t Mpool = (L + B - 1) / B;
-  if (Mpool > kMaxBlocks || T < 4 * QT) return false;
-  if (nseq > 1 && T % QT != 0) return false;   // tiles must not straddle sequences
-  return (int64_t)nseq * T * H < INT32_MAX;
+  return (Mpool + kMaxBlocks - 1) / kMaxBlocks * kMaxBlocks;
 }
 
-size_t route_tc_ws_bytes(int nseq, int T, int H) {
+bool route_tc_supported(int nseq, int T, int H, int64_t L, int B) {
+  if (H < 8 || H > 128 || (128 % H) != 0 || encode_fn() == nullptr) return false;
+  const int QT = 128 / H;
+  const int64_t mpad = route_tc_mpad(L, B);
+  if (mpad > 65536 || T < 4 * QT) return false;
+  if (nseq > 1 && T % QT != 0) return false;   // tiles must not straddle sequences
+  return (int64_t)nseq * T * H < INT32_MAX && (int64_t)nseq * mpad < INT32_MAX;
+}
+
+size_t route_tc_ws_bytes(int nseq, int T, int H, int64_t L, int B) {
+  (void)H;
   const size_t rows = (size_t)nseq * T;
-  return 2 * align256((size_t)nseq * kMaxBlocks * kHeadDim * 2) +
-         align256(rows * kHeadDim * 4) + align256(rows * H * 4);
+  // pooled keys hi + lo; the partial keys, padded by a tile's queries (the last tile's copy)
+  return 2 * align256((size_t)nseq * route_tc_mpad(L, B) * kHeadDim * 2) +
+         align256((rows + kMaxQT) * kHeadDim * 4);
 }
 
 cudaError_t launch_route_tc(const uint16_t* q, const float* w, const uint16_t* k,
@@ -380,25 +474,25 @@ cudaError_t launch_route_tc(const uint16_t* q, const float* w, const uint16_t* k
                             int* status, cudaStream_t st) {
   const int rows = nseq * T;
   const int Mpool = (int)((L + B - 1) / B);
+  const int mpad = (int)route_tc_mpad(L, B);
   char* c = reinterpret_cast<char*>(scratch);
   uint16_t* hi = reinterpret_cast<uint16_t*>(c);
-  c += align256((size_t)nseq * kMaxBlocks * kHeadDim * 2);
+  c += align256((size_t)nseq * mpad * kHeadDim * 2);
   uint16_t* lo = reinterpret_cast<uint16_t*>(c);
-  c += align256((size_t)nseq * kMaxBlocks * kHeadDim * 2);
+  c += align256((size_t)nseq * mpad * kHeadDim * 2);
   float* kpart = reinterpret_cast<float*>(c);
-  c += align256((size_t)rows * kHeadDim * 4);
-  float* Ebuf = E ? E : reinterpret_cast<float*>(c);
 
-  route_tc_split_kernel<<<nseq * kMaxBlocks, kHeadDim, 0, st>>>(k_pool, Mpool, hi, lo);
+  route_tc_split_kernel<<<nseq * mpad, kHeadDim, 0, st>>>(k_pool, Mpool, mpad, hi, lo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  route_tc_partial_kernel<<<rows, kHeadDim, 0, st>>>(k, pos, T, L, B, kpart, status);
+  route_tc_partial_kernel<<<(rows + kPartWarps - 1) / kPartWarps, 32 * kPartWarps, 0, st>>>(
+      k, pos, rows, T, L, B, kpart, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, thi, tlo;
   if (!make_map(&tq, q, (uint64_t)rows * H, kRows) ||
-      !make_map(&thi, hi, (uint64_t)nseq * kMaxBlocks, kMaxBlocks) ||
-      !make_map(&tlo, lo, (uint64_t)nseq * kMaxBlocks, kMaxBlocks))
+      !make_map(&thi, hi, (uint64_t)nseq * mpad, kMaxBlocks) ||
+      !make_map(&tlo, lo, (uint64_t)nseq * mpad, kMaxBlocks))
     return cudaErrorInvalidValue;
   RouteGeo g;
   g.T = T;
@@ -407,6 +501,7 @@ cudaError_t launch_route_tc(const uint16_t* q, const float* w, const uint16_t* k
   g.QT = 128 / H;
   g.L = L;
   g.tiles_per_seq = (T + g.QT - 1) / g.QT;
+  g.mpad = mpad;
   const int total_tiles = nseq * g.tiles_per_seq;
   e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes);
@@ -414,11 +509,8 @@ cudaError_t launch_route_tc(const uint16_t* q, const float* w, const uint16_t* k
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  route_tc_kernel<<<sms, kThreads, kSmemBytes, st>>>(tq, thi, tlo, q, w, kpart, pos, g, total_tiles,
-                                                     Ebuf, status);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  route_tc_select_kernel<<<(rows * 32 + 255) / 256, 256, 0, st>>>(Ebuf, rows, H, h, heads);
+  route_tc_kernel<<<sms, kThreads, kSmemBytes, st>>>(tq, thi, tlo, w, kpart, pos, g, total_tiles,
+                                                     h, heads, E, status);
   return cudaGetLastError();
 }
 

@@ -588,8 +588,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) topk_group_kernel(
   const uint64_t* src = cand + row * (int64_t)hist_groups(topk) * kGroupBuf + g * kGroupBuf;
   for (uint32_t i = t; i < cnt; i += kSelThreads) gathered[i] = src[i];
   __syncthreads();
+  const uint64_t* res = gathered;   // the counting sort leaves its result in place
   if (!group_sort_desc<kSelThreads>(gathered, cnt, sorted, buckets, blo, bhi, warp_sums, s_flag)) {
     // crowded buckets (many equal scores): bitonic sort of the group instead
+    res = sorted;
     int sortn = kSelThreads;
     while ((uint32_t)sortn < cnt) sortn <<= 1;
     for (int i = t; i < sortn; i += kSelThreads) sorted[i] = (uint32_t)i < cnt ? gathered[i] : 0ull;
@@ -604,7 +606,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) topk_group_kernel(
     }
   }
   for (uint32_t i = t; i < cnt && start + i < target; i += kSelThreads) {
-    const uint64_t v = sorted[i];
+    const uint64_t v = res[i];
     const int64_t o = row * topk + start + i;
     idx[o] = (int32_t)(~(uint32_t)(v & 0xffffffffu));
     if (vals) vals[o] = key_score((uint32_t)(v >> 32));
@@ -860,7 +862,45 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     __syncthreads();
   }
   const bool fits = C <= (uint32_t)CAP;
+  // Candidates go to cin[0 .. C); the sort uses cscr as scratch.  The one-pass compaction:
+  // warp w takes the row's 32-key steps w, w + kWarps, ... (an even sample of the row) and
+  // appends its candidates to its own region of CAP / kWarps slots of cand; the regions are
+  // then packed into the (dead) key space.  A region that overflows sends the row through
+  // the two-pass compaction (count per warp slice, block scan, ballot ranks).
+  uint64_t* cin = cand;
+  uint64_t* cscr = sorted;
+  bool packed = false;
   if (fits) {
+    constexpr uint32_t kReg = (uint32_t)CAP / kWarps;
+    uint32_t wc = 0;
+#pragma unroll 4
+    for (int e0 = warp * 32; e0 < n; e0 += 32 * kWarps) {
+      const int e = e0 + lane;
+      const uint32_t key = e < n ? keys[e] : 0u;
+      const bool take = e < n && key >= kcut;
+      const uint32_t m = __ballot_sync(0xffffffffu, take);
+      const uint32_t r = wc + __popc(m & below);
+      if (take && r < kReg) cand[warp * kReg + r] = compose(key, e);
+      wc += __popc(m);
+    }
+    if (lane == 0) warp_sums[warp] = wc;
+    if (!__syncthreads_or(wc > kReg ? 1 : 0)) {
+      uint32_t pre = 0, tot = 0;
+#pragma unroll
+      for (int w2 = 0; w2 < kWarps; ++w2) {
+        const uint32_t x = warp_sums[w2];
+        if (w2 < warp) pre += x;
+        tot += x;
+      }
+      for (uint32_t i = lane; i < wc; i += 32) sorted[pre + i] = cand[warp * kReg + i];
+      C = tot;
+      cin = sorted;
+      cscr = cand;
+      packed = true;
+    }
+    __syncthreads();   // warp_sums is reused below
+  }
+  if (fits && !packed) {
     if ((select && !given) || refined) {   // count this lane's candidates (else counted above)
       cnt = 0;
 #pragma unroll 4
@@ -882,7 +922,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       if (take && r < (uint32_t)CAP) cand[r] = compose(key, e);   // (a histogram that
       p += __popc(m);                                            //  disagrees cannot overflow)
     }
-  } else {
+  } else if (!fits) {
     // crowded cutoff bin: exact threshold by a radix select over the resident keys, then
     // exactly `target` pairs (above the threshold, then equal ones in index order)
     uint32_t prefix = 0, mask = 0, kneed = target;
@@ -966,13 +1006,20 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     block_minmax<NT>(lo_dummy, btop, red);
   }
   __syncthreads();
-  // keys are dead from here on: their space holds the sorted pairs
-  if (C > 0 && !group_sort_adaptive<NT>(cand, C, sorted, hist,
+  // keys are dead from here on: their space is the sort's scratch.  The per-bin counts of
+  // the candidates are the histogram's when every key of bins [cut, btop] is a candidate.
+  const uint32_t* bin_counts = (select && fits && !refined) ? hist : nullptr;
+  const uint64_t* res = cin;   // the counting sort leaves its result in place
+  if (C > 0 && !group_sort_adaptive<NT>(cin, C, cscr, hist,
                                reinterpret_cast<uint8_t*>(rbuf) + RC::kAuxOff, cut, btop,
-                               warp_sums, s_flag, s_nsub)) {
+                               warp_sums, s_flag, s_nsub, bin_counts)) {
+    res = sorted;
     int sortn = NT;
     while ((uint32_t)sortn < C) sortn <<= 1;
-    for (int i = t; i < sortn; i += NT) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
+    if (cin == cand)
+      for (int i = t; i < sortn; i += NT) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
+    else
+      for (int i = (int)C + t; i < sortn; i += NT) sorted[i] = 0ull;
     __syncthreads();
     row_bitonic<NT, RC::kEMax>(sorted, sortn);
   }
@@ -986,7 +1033,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       id[u] = -1;
       key[u] = 0u;
       if (i < topk && (uint32_t)i < target) {
-        const uint64_t v = sorted[i];
+        const uint64_t v = res[i];
         const int32_t e = (int32_t)(~(uint32_t)(v & 0xffffffffu));   // position in the row
         id[u] = imap ? imap[e] : e;
         key[u] = (uint32_t)(v >> 32);

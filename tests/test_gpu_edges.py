@@ -61,6 +61,12 @@ CASES = {
     # many queries per sequence: tensor-core router and query-block scorer
     "blocks_two_seqs_H16": dict(nseq=2, T=64, L=1000, H=16, h=4, topk=64, kprime=128),
     "blocks_H64_B32": dict(nseq=1, T=40, L=3000, H=64, h=8, B=32, topk=128, kprime=256),
+    # tensor-core router shapes: 16 queries per tile with a partial last tile, 4 per tile
+    # over two sequences, and a prefix beyond 16K (512 pooled blocks)
+    "route_tc_H8_partial_tile": dict(nseq=1, T=100, L=3000, H=8, h=3, topk=64, kprime=128),
+    "route_tc_H32_two_seqs": dict(nseq=2, T=64, L=2000, H=32, h=8, B=32, topk=64, kprime=128),
+    "prefill_32k_prefix": dict(nseq=1, T=64, L=32768, H=64, h=8, B=64, topk=2048,
+                               kprime=4096),
 }
 
 

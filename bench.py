@@ -141,15 +141,19 @@ def block_form(wl) -> bool:
 def misa_step_launches(wl) -> int:
     """Kernels one MISA step launches, following the library's dispatch: pooling, the router
     (one kernel, or three on tcgen05 for many queries per sequence), the scorer's
-    gather/offsets kernel and the scorer, then the top-k: one kernel, except decode rows
-    longer than 40960 scores (or k > 3072) with the scorer's histogram, which take a
-    scatter and a group kernel (and an overflow kernel above k = 4096)."""
+    gather/offsets kernel and the scorer, then the top-k: one kernel, except histogrammed
+    rows longer than 40960 scores or with k > 3072, which take a scatter and a group kernel
+    (and an overflow kernel above k = 4096); rows of several queries per sequence longer
+    than 16384 scores first take a histogram pass."""
     qt = 128 // wl.H if (128 % wl.H == 0 and wl.H >= 8) else 0
     route_tc = qt > 0 and wl.T >= 4 * qt and (wl.nseq == 1 or wl.T % qt == 0)
     n = 1 + (3 if route_tc else 1)
     n += 2
     hist_path = wl.rows <= 1024 and wl.L >= 8192 and not block_form(wl)
-    if hist_path and not (wl.L <= 40960 and wl.topk <= 3072):
+    hist_kernel = wl.rows <= 1024 and wl.L > 16384 and block_form(wl)
+    if hist_kernel:
+        n += 1
+    if (hist_path or hist_kernel) and not (wl.L <= 40960 and wl.topk <= 3072):
         n += 2 + (wl.topk > 4096)
     else:
         n += 1

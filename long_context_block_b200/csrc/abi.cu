@@ -39,10 +39,7 @@ int check_topk(int topk) {
 size_t route_ws(int nseq, int T, int H, int64_t L, int B) {
   if (route_tc_supported(nseq, T, H, L, B))
     return kStatusBytes + route_tc_ws_bytes(nseq, T, H, L, B);
-  const int64_t M = (L + B - 1) / B;
-  const int64_t nchunk = (M + kRouteChunk - 1) / kRouteChunk;
-  return kStatusBytes + align256((size_t)nseq * T * nchunk * H * sizeof(float)) +
-         align256((size_t)nseq * T * sizeof(int));
+  return kStatusBytes;   // the cluster router needs no scratch
 }
 // Rows up to this count whose length reaches kHistPathMinLen use the histogram-filtered
 // top-k, fed by a score histogram built in the tensor-core scorer's epilogue.
@@ -53,12 +50,20 @@ bool hist_path(int nseq, int T, int64_t L, int nh) {
   return (int64_t)nseq * T <= kHistPathMaxRows && L >= kHistPathMinLen &&
          !score_tc_block_form(nh, T);
 }
+// Rows of several queries per sequence longer than the row top-k holds (16384 scores): the
+// histogram comes from a separate pass over the scores instead of the scorer's epilogue.
+constexpr int64_t kHistKernelMinLen = 16385;
+bool hist_kernel_path(int nseq, int T, int64_t L, int nh) {
+  return (int64_t)nseq * T <= kHistPathMaxRows && L >= kHistKernelMinLen &&
+         score_tc_block_form(nh, T);
+}
 
 size_t score_ws(int nseq, int T, int64_t L, int nh, int topk) {
   const int64_t rows = (int64_t)nseq * T;
   return kStatusBytes + align256((size_t)rows * L * sizeof(float)) +
          score_tc_ws_bytes(nseq, T, nh) +
-         (hist_path(nseq, T, L, nh) ? topk_hist_ws_bytes(rows, topk) : 0);
+         (hist_path(nseq, T, L, nh) || hist_kernel_path(nseq, T, L, nh)
+              ? topk_hist_ws_bytes(rows, topk) : 0);
 }
 size_t dagger_ws(int nseq, int T, int H, int kprime) {
   const size_t rows = (size_t)nseq * T;
@@ -146,11 +151,7 @@ int misa_route_heads(const uint16_t* q, const float* w, const uint16_t* k, const
   if (route_tc_supported(nseq, T, H, L, B))
     return cuda_status(launch_route_tc(q, w, k, k_pool, pos, nseq, T, H, L, B, h, heads, E,
                                        ws_region(ws, 0), status_word(ws), (cudaStream_t)stream));
-  const int nchunk = (int)((M + kRouteChunk - 1) / kRouteChunk);
-  const size_t part_bytes = align256(rows * nchunk * H * sizeof(float));
   return cuda_status(launch_route(q, w, k, k_pool, pos, nseq, T, H, L, B, h, heads, E,
-                                  reinterpret_cast<float*>(ws_region(ws, 0)), nchunk,
-                                  reinterpret_cast<int*>(ws_region(ws, part_bytes)),
                                   status_word(ws), (cudaStream_t)stream));
 }
 
@@ -175,16 +176,18 @@ static int score_topk_common(const uint16_t* q, const float* w, const uint16_t* 
   if (score_tc_supported(nseq, T, nh, L)) {
     const size_t sc_bytes = align256(rows * L * sizeof(float));
     void* tc_scratch = ws_region(ws, sc_bytes);
-    if (hist_path(nseq, T, L, nh)) {
+    if (hist_path(nseq, T, L, nh) || hist_kernel_path(nseq, T, L, nh)) {
       char* hp = ws_region(ws, sc_bytes + score_tc_ws_bytes(nseq, T, nh));
       const size_t hb = align256(rows * kScoreHistBins * 4);
-      const size_t gb = align256(rows * 16 * 4);
       uint32_t* hist = reinterpret_cast<uint32_t*>(hp);
       uint32_t* gcount = reinterpret_cast<uint32_t*>(hp + hb);
-      uint64_t* cand = reinterpret_cast<uint64_t*>(hp + hb + gb);
-      MISA_TRY(cuda_status(cudaMemsetAsync(hist, 0, hb + gb, st)));
+      uint64_t* cand = reinterpret_cast<uint64_t*>(hp + topk_hist_zero_bytes(rows));
+      // the scorer's prep kernel zeroes the histogram and the group counts
       MISA_TRY(cuda_status(launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, sc, L,
-                                           tc_scratch, status, hist, st)));
+                                           tc_scratch, status, hist, st, nullptr, nullptr,
+                                           nullptr, topk_hist_zero_bytes(rows))));
+      if (!hist_path(nseq, T, L, nh))
+        MISA_TRY(cuda_status(launch_build_hist(sc, L, pos, L, (int)rows, hist, st)));
       return cuda_status(launch_topk_hist(sc, L, pos, L, hist, cand, gcount, (int)rows, topk, idx,
                                           vals, status, st));
     }

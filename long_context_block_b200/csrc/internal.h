@@ -54,12 +54,12 @@ constexpr int kRouteChunk = 32;
 cudaError_t launch_pool_mean(const uint16_t* k, int nseq, int64_t L, int B, float* k_pool,
                              cudaStream_t st, int64_t s_begin = 0, int64_t s_end = -1);
 
-// K2 -- router: partial head energies per chunk of blocks, then E and top-h by the
-// last CTA of each row (route.cu).  `counters` is rows ints of scratch (zeroed here).
+// K2 -- router (route.cu): a thread-block cluster per query row sums the head energies
+// over chunks of the prefix's pooled blocks, then E and the top-h.  No scratch.
 cudaError_t launch_route(const uint16_t* q, const float* w, const uint16_t* k,
                          const float* k_pool, const int32_t* pos, int nseq, int T, int H,
-                         int64_t L, int B, int h, int32_t* heads, float* E, float* partial,
-                         int nchunk, int* counters, int* status, cudaStream_t st);
+                         int64_t L, int B, int h, int32_t* heads, float* E, int* status,
+                         cudaStream_t st);
 
 // K2 in block-score mode (route.cu), for the HISA-style filter: G[row, b] = sum_j
 // w[row,j] * ReLU(q[row,j] . kp_b) for the blocks b < M_t of each query's prefix (row stride
@@ -106,8 +106,10 @@ cudaError_t launch_score_simt(const uint16_t* q, const float* w, const uint16_t*
 bool score_tc_supported(int nseq, int T, int nh, int64_t L, int64_t span = 0);
 bool score_tc_block_form(int nh, int T);
 size_t score_tc_ws_bytes(int nseq, int T, int nh, bool gather = false);
-//   hist (nullable, zeroed by the caller): per-row kScoreHistBins-bin histogram of the
-//   written scores' keys, accumulated in the epilogue (prefix decode form only).
+//   hist (nullable): per-row kScoreHistBins-bin histogram of the written scores' keys,
+//   accumulated in the epilogue (prefix decode form only; in the other forms it is left for
+//   launch_build_hist); the scorer's prep kernel first zeroes hist_zero_bytes bytes (a
+//   multiple of 16) from hist in every form.
 //   gather_ids / gather_len (both or neither): row r scores the gather_len[r] tokens
 //   gather_ids[r * out_stride + i] (each in [0, L)) into out[r * out_stride + i]; every
 //   row takes the decode form and its keys are fetched four rows per TMA gather.
@@ -125,7 +127,8 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
                             int* status, uint32_t* hist, cudaStream_t st,
                             const int32_t* gather_ids = nullptr,
                             const int32_t* gather_len = nullptr,
-                            const WaitProbe* test_probe = nullptr);
+                            const WaitProbe* test_probe = nullptr,
+                            size_t hist_zero_bytes = 0);
 
 // K5 -- per-row top-k selection (topk.cu).
 //   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.
@@ -139,15 +142,21 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
 // shared memory (up to 40960 scores, k <= 3072) are selected by one CTA per row that takes
 // the cutoff bin from the histogram; longer rows split the bins at or above the cutoff
 // into groups of output positions: a scatter pass appends every candidate to its group's
-// buffer and one CTA per group sorts and writes it.  hist: rows x kScoreHistBins (filled
-// by the scorer); gcount: rows x 16 (zeroed by the caller, directly after hist); cand:
-// topk_hist_ws_bytes layout.
+// buffer and one CTA per group sorts and writes it.  hist: rows x kScoreHistBins;
+// gcount: rows x 16 (zeroed, directly after hist); cand: topk_hist_ws_bytes layout.
 cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
                              const uint32_t* hist, uint64_t* cand, uint32_t* gcount, int rows,
                              int topk, int32_t* idx, float* vals, int* status, cudaStream_t st);
+// The score histogram (kScoreHistBins bins per row, zeroed by the caller) of rows that the
+// scorer did not histogram (topk.cu).  rows <= 65535.
+cudaError_t launch_build_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
+                              int rows, uint32_t* hist, cudaStream_t st);
 // Scratch of the histogram path: histogram, group counts, group buffers (ceil(topk / 1024)
 // groups of 8192 pairs per row), each region 256-aligned.
 size_t topk_hist_ws_bytes(int64_t rows, int topk);
+// Bytes at the start of that scratch which must be zero before the scores are histogrammed
+// (the histogram and the group counts).
+size_t topk_hist_zero_bytes(int64_t rows);
 
 // Power-of-two length of the shared-memory sort buffer for `topk` entries (topk.cu).
 int topk_sort_size(int topk);

@@ -15,13 +15,15 @@
 // MMAs reproduce the fp32 products to about 2^-16 relative.  Accumulators live in TMEM
 // (N = the item's largest full-block count within its chunk, rounded up to 16).
 //
-// Epilogue: 8 warps, two per TMEM lane quarter; the two warps of a quarter split the
-// accumulator columns (masked to each row's own causal block count) and the partial-block
-// dot product (64 dimensions each), which reads the query rows from the tile's A stage
-// (the stage is released by the epilogue, not by the MMA) and the tile's partial pooled
-// keys from a shared-memory copy loaded with the A tile.  The halves are combined through
-// shared memory, E is written (when asked for), and every row ranks its head among its
-// query's H energies to write the top-h heads.
+// Epilogue: two groups of 4 warps (one per TMEM lane quarter); group g serves the tiles
+// t0 + g, t0 + g + 2, ... with its own pair of 128-column accumulators, so the two groups'
+// per-tile latency chains overlap and the MMAs of a group's next item run while it reads the
+// current one.  Each warp owns 32 (query, head) rows of its tile: the partial-block dot
+// product reads the query row from the tile's A stage (released by the epilogue, not by the
+// MMA) and the tile's partial pooled keys from a shared-memory copy loaded with the A tile;
+// then the row's ReLU sum over its causal block count, E (written when asked for), and a
+// rank of the row's head among its query's H energies for the top-h heads.  The tile's
+// per-row inputs (prefix lengths, |w|) are loaded one group tile ahead.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -39,14 +41,18 @@ constexpr int kRows = 128;                          // (query, head) rows per ti
 constexpr int kATileBytes = kRows * kHeadDim * 2;   // 32 KB
 constexpr int kAHalf = kATileBytes / 2;
 constexpr int kMaxBlocks = 256;                     // pooled keys per chunk (one resident)
+constexpr int kItemBlocks = 128;                    // accumulator columns of one MMA item
 constexpr int kBBytes = kMaxBlocks * kHeadDim * 2;  // 64 KB per part (hi or lo)
 constexpr int kBHalf = kBBytes / 2;
 constexpr int kMaxQT = 16;                          // queries per tile (H >= 8)
 constexpr int kKpBytes = kMaxQT * kHeadDim * 4;     // partial pooled keys of a tile (fp32)
-constexpr int kStages = 2;
-constexpr int kAcc = 2;
-constexpr int kCols = 512;
-constexpr int kEpiWarps = 8;
+constexpr int kGroups = 2;                          // epilogue groups
+constexpr int kStages = kGroups;                    // stage s holds the tiles group s serves
+constexpr int kAccPerGroup = 2;
+constexpr int kAcc = kGroups * kAccPerGroup;
+constexpr int kCols = kAcc * kItemBlocks;           // 512
+constexpr int kGroupThreads = 128;
+constexpr int kEpiWarps = kGroups * 4;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr long long kWaitCycles = 4000000000LL;
@@ -54,14 +60,14 @@ constexpr long long kWaitCycles = 4000000000LL;
 constexpr int kStageBase = 0;
 constexpr int kBBase = kStages * kATileBytes;         // hi then lo
 constexpr int kKpBase = kBBase + 2 * kBBytes;
-constexpr int kEsBase = kKpBase + kStages * kKpBytes;  // E of the tile's rows
-constexpr int kXBase = kEsBase + kRows * 4;            // second half's sums: [2][kRows]
-constexpr int kBarBase = kXBase + 2 * kRows * 4;
+constexpr int kEsBase = kKpBase + kStages * kKpBytes;  // E of a tile's rows: [group][2][kRows]
+constexpr int kBarBase = kEsBase + kGroups * 2 * kRows * 4;
 // full[S], empty[S], bfull, bempty, accfull[A], accempty[A], drain
 constexpr int kNumBars = 2 * kStages + 2 + 2 * kAcc + 1;
 constexpr int kMiscBase = kBarBase + kNumBars * 8;
 constexpr int kSmemBytes = kMiscBase + 16 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kStages == kGroups && kGroups == 2 && kMaxBlocks == 2 * kItemBlocks, "tile-to-group map");
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
   volatile int never = 0;
@@ -75,8 +81,28 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-__device__ __forceinline__ void epi_bar() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+__device__ __forceinline__ void group_bar(int grp) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(kGroupThreads) : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes: two loads, one wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr), "r"(taddr + 16u)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 struct RouteGeo {
@@ -95,9 +121,15 @@ __device__ __forceinline__ int tile_blocks(const int32_t* pos, const RouteGeo& g
     mf = max(mf, prefix_len(pos, (int64_t)n * g.T + ta + qq, g.L, nullptr) / g.B);
   return mf;
 }
-// MMA items of a tile whose queries reach mf full blocks, and the chunk of its k-th item.
+// Chunks of pooled keys a tile whose queries reach mf full blocks visits, and the chunk of
+// its k-th visit.  Inside chunk c the tile makes one MMA item per 128-block half that holds
+// full blocks (item_present(c, sub, mf)); a tile without full blocks makes one empty item.
 __device__ __forceinline__ int tile_items(int mf) { return max(1, (mf + kMaxBlocks - 1) / kMaxBlocks); }
 __device__ __forceinline__ int item_chunk(int i, int k, int nc) { return (i & 1) ? nc - 1 - k : k; }
+__device__ __forceinline__ bool item_present(int c, int sub, int mf) {
+  const int b0 = c * kMaxBlocks + sub * kItemBlocks;
+  return b0 < mf || (mf == 0 && b0 == 0);
+}
 
 __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
@@ -123,13 +155,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kEpiWarps);   // the MMAs' commit and every epilogue warp
+      mbar_init(&empty[s], 1 + 4);   // the MMAs' commit and the serving group's warps
     }
     mbar_init(bfull, 1);
     mbar_init(bempty, 1);
     for (int a = 0; a < kAcc; ++a) {
       mbar_init(&accfull[a], 1);
-      mbar_init(&accempty[a], kEpiThreads);
+      mbar_init(&accempty[a], kGroupThreads);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -194,12 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t smem0 = smem_u32(base);
-      int it = 0, acc_it = 0, bseen = 0;
+      int it = 0, bseen = 0;
+      int uses0 = 0, uses1 = 0;   // items issued for each group's accumulator pair
       int64_t cur_key = -1;
       bool ok = true;
       for (int i = t0; i < t1 && ok; ++i) {
         const int n = i / g.tiles_per_seq;
-        const int s = it % kStages;
+        const int s = it % kStages, grp = it % kGroups;
         if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, status, kWaitCycles)) break;
         const int mf = tile_blocks(pos, g, i);
         const int nc = tile_items(mf);
@@ -215,33 +248,39 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
             ++bseen;
             cur_key = key;
           }
-          const int acc = acc_it % kAcc;
-          if (!mbar_wait(&accempty[acc], ((acc_it / kAcc) & 1) ^ 1, abort_flag, status,
-                         kWaitCycles)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int nb = min(max(mf - c * kMaxBlocks, 0), kMaxBlocks);
-          const int N = (nb + 15) & ~15;
-          if (N > 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, N);
-            const uint32_t aaddr = smem0 + kStageBase + s * kATileBytes;
-            const uint32_t d = tmem_base + (uint32_t)(acc * 256);
+          for (int sub = 0; sub < kMaxBlocks / kItemBlocks && ok; ++sub) {
+            if (!item_present(c, sub, mf)) continue;
+            const int u = grp ? uses1++ : uses0++;
+            const int acc = grp * kAccPerGroup + (u % kAccPerGroup);
+            if (!mbar_wait(&accempty[acc], ((u / kAccPerGroup) & 1) ^ 1, abort_flag, status,
+                           kWaitCycles)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int b0 = c * kMaxBlocks + sub * kItemBlocks;
+            const int nb = min(max(mf - b0, 0), kItemBlocks);
+            const int N = (nb + 15) & ~15;
+            if (N > 0) {
+              const uint32_t idesc = idesc_bf16_f32(128, N);
+              const uint32_t aaddr = smem0 + kStageBase + s * kATileBytes;
+              const uint32_t d = tmem_base + (uint32_t)(acc * kItemBlocks);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-              const uint32_t baddr = smem0 + kBBase + part * kBBytes;
+              for (int part = 0; part < 2; ++part) {
+                // rows sub * 128 .. of the resident chunk (whole 1 KB swizzle atoms)
+                const uint32_t baddr =
+                    smem0 + kBBase + part * kBBytes + sub * kItemBlocks * 128;
 #pragma unroll
-              for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-                const uint32_t ao = (kk >> 2) * kAHalf + (kk & 3) * 32;
-                const uint32_t bo = (kk >> 2) * kBHalf + (kk & 3) * 32;
-                mma_bf16(d, desc_kmajor_sw128(aaddr + ao), desc_kmajor_sw128(baddr + bo), idesc,
-                         (part | kk) ? 1u : 0u);
+                for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+                  const uint32_t ao = (kk >> 2) * kAHalf + (kk & 3) * 32;
+                  const uint32_t bo = (kk >> 2) * kBHalf + (kk & 3) * 32;
+                  mma_bf16(d, desc_kmajor_sw128(aaddr + ao), desc_kmajor_sw128(baddr + bo),
+                           idesc, (part | kk) ? 1u : 0u);
+                }
               }
             }
+            mma_commit(&accfull[acc]);
           }
-          mma_commit(&accfull[acc]);
-          ++acc_it;
         }
         if (!ok) break;
         mma_commit(&empty[s]);   // the tile's A stage, once all its items' MMAs are done
@@ -256,97 +295,116 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     tmem_dealloc(tmem_base, kCols);
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9)
-    const int e = warp - 2;
-    const int grp = e >> 2;              // 0: even column chunks, dims 0-63; 1: odd, 64-127
+    const int grp = (warp - 2) >> 2;     // group: tiles t0 + grp, t0 + grp + 2, ...
     const int quarter = warp & 3;        // TMEM lanes this warp may read
     const int r = quarter * 32 + lane;   // row of the tile
     const int qq = r / g.H, j = r % g.H;
-    float* Es = reinterpret_cast<float*>(base + kEsBase);
-    float* xsum = reinterpret_cast<float*>(base + kXBase);
-    float* xdot = xsum + kRows;
-    // Every epilogue warp walks every tile and meets both named barriers of each, whatever
-    // happens; after a failed (bounded) wait a warp only skips the work.
+    float* Es2 = reinterpret_cast<float*>(base + kEsBase) + grp * 2 * kRows;
+    // Per-row inputs of tile i: lane l < QT reads query l's prefix length (the tile's
+    // largest full-block count is their maximum), every lane its own |w|.
+    auto load_meta = [&](int i, int& Pl, float& wabs) {
+      const int n = i / g.tiles_per_seq;
+      const int ta = (i % g.tiles_per_seq) * g.QT;
+      Pl = (lane < g.QT && ta + lane < g.T)
+               ? prefix_len(pos, (int64_t)n * g.T + ta + lane, g.L, nullptr) : 0;
+      const int tq = ta + qq;
+      wabs = fabsf(w[((int64_t)n * g.T + (tq < g.T ? tq : 0)) * g.H + j]);
+    };
+    // Every epilogue warp of a group walks every tile of the group and meets the group
+    // barrier of each, whatever happens; after a failed (bounded) wait a warp only skips
+    // the work.
     bool ok = true;
-    int it = 0, acc_it = 0;
-    for (int i = t0; i < t1; ++i, ++it) {
+    int uses = 0, gt = 0;
+    int Pl_next = 0;
+    float w_next = 0.f;
+    if (t0 + grp < t1) load_meta(t0 + grp, Pl_next, w_next);
+    for (int i = t0 + grp, it = grp; i < t1; i += kGroups, it += kGroups, ++gt) {
       const int s = it % kStages;
       const int n = i / g.tiles_per_seq;
       const int ta = (i % g.tiles_per_seq) * g.QT;
       const int tq = ta + qq;
       const bool valid = tq < g.T;
       const int64_t qrow = (int64_t)n * g.T + (valid ? tq : 0);
-      const int P = prefix_len(pos, qrow, g.L, nullptr);
+      const int Pl = Pl_next;
+      const float wabs = w_next;
+      if (i + kGroups < t1) load_meta(i + kGroups, Pl_next, w_next);   // one group tile ahead
+      int mf = Pl / g.B;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mf = max(mf, __shfl_xor_sync(0xffffffffu, mf, o));
+      const int P = __shfl_sync(0xffffffffu, Pl, valid ? qq : 0);   // qq < QT <= 16
       const int mfull = P / g.B;
       const int M = (P + g.B - 1) / g.B;
-      const float wabs = fabsf(w[qrow * g.H + j]);
-      const int nc = tile_items(tile_blocks(pos, g, i));
-      float sum = 0.f, dot = 0.f;
-      // the partial last block first: its half of q . kpart (64 dimensions) reads the query
-      // row from the tile's A stage and the partial keys copied with it, as soon as they
-      // landed, and then releases the stage
+      const int nc = tile_items(mf);
+      // the partial last block: q . kpart over 128 dimensions, reading the query row from
+      // the tile's A stage and the partial keys copied with it, then releasing the stage
+      float dot = 0.f;
       if (ok && !warp_wait(&full[s], (it / kStages) & 1, abort_flag, status)) ok = false;
       if (ok && M > mfull) {
-        const uint8_t* arow = base + kStageBase + s * kATileBytes + grp * kAHalf + r * 128;
-        const float4* kv = reinterpret_cast<const float4*>(base + kKpBase + s * kKpBytes +
-                                                           (qq * kHeadDim + grp * 64) * 4);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {   // 16-byte chunk c of the row (128-byte swizzle)
-          const uint4 x = *reinterpret_cast<const uint4*>(arow + ((c ^ (r & 7)) << 4));
-          const float4 a = kv[2 * c], b = kv[2 * c + 1];
-          dot = fmaf(bf16lo(x.x), a.x, dot); dot = fmaf(bf16hi(x.x), a.y, dot);
-          dot = fmaf(bf16lo(x.y), a.z, dot); dot = fmaf(bf16hi(x.y), a.w, dot);
-          dot = fmaf(bf16lo(x.z), b.x, dot); dot = fmaf(bf16hi(x.z), b.y, dot);
-          dot = fmaf(bf16lo(x.w), b.z, dot); dot = fmaf(bf16hi(x.w), b.w, dot);
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint8_t* arow = base + kStageBase + s * kATileBytes + hf * kAHalf + r * 128;
+          const float4* kv = reinterpret_cast<const float4*>(base + kKpBase + s * kKpBytes +
+                                                             (qq * kHeadDim + hf * 64) * 4);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {   // 16-byte chunk c of the row (128-byte swizzle)
+            const uint4 x = *reinterpret_cast<const uint4*>(arow + ((c ^ (r & 7)) << 4));
+            const float4 a = kv[2 * c], b = kv[2 * c + 1];
+            dot = fmaf(bf16lo(x.x), a.x, dot); dot = fmaf(bf16hi(x.x), a.y, dot);
+            dot = fmaf(bf16lo(x.y), a.z, dot); dot = fmaf(bf16hi(x.y), a.w, dot);
+            dot = fmaf(bf16lo(x.z), b.x, dot); dot = fmaf(bf16hi(x.z), b.y, dot);
+            dot = fmaf(bf16lo(x.w), b.z, dot); dot = fmaf(bf16hi(x.w), b.w, dot);
+          }
         }
       }
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(&empty[s]);   // this warp is done with the stage
-      for (int k = 0; k < nc; ++k, ++acc_it) {   // the tile's items, one chunk each
-        const int acc = acc_it % kAcc;
-        // this row's full blocks inside the item's chunk, and the warp's largest count
-        const int mrow = min(max(mfull - item_chunk(i, k, nc) * kMaxBlocks, 0), kMaxBlocks);
-        int mwarp = mrow;
+      float sum = 0.f;
+      for (int k = 0; k < nc; ++k) {   // the tile's items, in the MMA warp's order
+        const int c = item_chunk(i, k, nc);
+#pragma unroll 1
+        for (int sub = 0; sub < kMaxBlocks / kItemBlocks; ++sub) {
+          if (!item_present(c, sub, mf)) continue;
+          const int acc = grp * kAccPerGroup + (uses % kAccPerGroup);
+          const uint32_t par = (uses / kAccPerGroup) & 1;
+          ++uses;
+          // this row's full blocks inside the item, and the warp's largest count
+          const int mrow = min(max(mfull - (c * kMaxBlocks + sub * kItemBlocks), 0), kItemBlocks);
+          int mwarp = mrow;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-          mwarp = max(mwarp, __shfl_xor_sync(0xffffffffu, mwarp, o));
-        if (ok && !warp_wait(&accfull[acc], (acc_it / kAcc) & 1, abort_flag, status)) ok = false;
-        if (ok) {
-          tc_fence_after();
-          const uint32_t taddr =
-              tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
-          for (int c0 = 16 * grp; c0 < mwarp; c0 += 32) {
-            float v[16];
-            tmem_ld16(taddr + c0, v);
-            if (c0 + 16 <= mrow) {
+          for (int o = 16; o > 0; o >>= 1)
+            mwarp = max(mwarp, __shfl_xor_sync(0xffffffffu, mwarp, o));
+          if (ok && !warp_wait(&accfull[acc], par, abort_flag, status)) ok = false;
+          if (ok) {
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                   (uint32_t)(acc * kItemBlocks);
+            for (int c0 = 0; c0 < mwarp; c0 += 32) {
+              float v[32];
+              tmem_ld32(taddr + c0, v);
+              if (c0 + 32 <= mrow) {
 #pragma unroll
-              for (int c = 0; c < 16; ++c) sum += fmaxf(v[c], 0.f);
-            } else {
+                for (int cc = 0; cc < 32; ++cc) sum += fmaxf(v[cc], 0.f);
+              } else {
 #pragma unroll
-              for (int c = 0; c < 16; ++c)
-                if (c0 + c < mrow) sum += fmaxf(v[c], 0.f);
+                for (int cc = 0; cc < 32; ++cc)
+                  if (c0 + cc < mrow) sum += fmaxf(v[cc], 0.f);
+              }
             }
+            tc_fence_before();
+            mbar_arrive(&accempty[acc]);
           }
-          tc_fence_before();
-          mbar_arrive(&accempty[acc]);
         }
       }
-      if (grp == 1) {
-        xsum[r] = sum;
-        xdot[r] = dot;
-      }
-      epi_bar();
-      if (grp == 0) {
-        const float tot = sum + xsum[r] + (M > mfull ? fmaxf(dot + xdot[r], 0.f) : 0.f);
-        const float ev = wabs * tot / (float)M;
-        Es[r] = ev;
-        if (ok && valid && E) E[qrow * g.H + j] = ev;
-      }
-      epi_bar();
+      float* Es = Es2 + (gt & 1) * kRows;   // alternate buffers: one group barrier per tile
+      const float tot = sum + (M > mfull ? fmaxf(dot, 0.f) : 0.f);
+      const float ev = wabs * tot / (float)M;
+      Es[r] = ev;
+      if (ok && valid && E) E[qrow * g.H + j] = ev;
+      group_bar(grp);
       // top-h heads: each row (one head of one query) counts the heads of its query that
       // come before it (larger E, or equal E and a lower index) and writes its own index at
       // that rank when the rank is below h
-      if (grp == 0 && ok && valid) {   // H is a multiple of 8: four energies per load
-        const float ev = Es[r];
+      if (ok && valid) {   // H is a multiple of 8: four energies per load
         const float4* eq = reinterpret_cast<const float4*>(Es + qq * g.H);
         int rank = 0;
         for (int j4 = 0; j4 < g.H / 4; ++j4) {

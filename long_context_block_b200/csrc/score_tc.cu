@@ -20,7 +20,7 @@
 //
 // Warp roles: warp 0 TMA producer (ring of 32 KB key tiles, each two 64-column boxes with
 // the 128-byte swizzle; per unit the q tile and its weights); warp 1 MMA issuer (one
-// thread) and TMEM owner; the epilogue warps (4 in decode form, 8 in block form) read
+// thread) and TMEM owner; the epilogue warps (4 in decode form, 8 or 16 in block form) read
 // their TMEM lane quarter with tcgen05.ld.  The grid is persistent (one CTA per SM); the
 // units' key tiles are laid end to end and every CTA takes a contiguous range of them,
 // so long and short units balance.  Every wait is bounded: on expiry the kernel records
@@ -56,7 +56,9 @@ constexpr int kIdAhead = 4;                                 // gather ids loaded
 template <int HS, int QB>
 struct Cfg {
   static constexpr int N = HS * QB;
-  static constexpr int kEpiWarps = QB == 1 ? 4 : 8;
+  // full-width blocks (N = 256) whose warps still cover whole queries take 16 epilogue warps
+  // (64 columns each), so the epilogue keeps up with the MMA; narrower blocks take 8
+  static constexpr int kEpiWarps = QB == 1 ? 4 : (HS * QB == 256 && HS <= 64 ? 16 : 8);
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kAcc = N <= 32 ? 8 : (N <= 64 ? 4 : 2);
   static constexpr int kAccStride = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
@@ -499,10 +501,13 @@ __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
     const uint16_t* __restrict__ q, const float* __restrict__ w, const int32_t* __restrict__ heads,
     int hsel, int H, int HS, Units geo, const int32_t* __restrict__ pos, int units, int64_t L,
     const int32_t* __restrict__ glen, int gmax, uint4* __restrict__ qg, float* __restrict__ wg,
-    int32_t* __restrict__ tile_off, int* status) {
+    int32_t* __restrict__ tile_off, int* status, uint4* __restrict__ zero, int64_t zero16) {
   pdl_prologue();
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
+  // zero the scorer's histogram scratch (zero16 16-byte words), spread over all blocks
+  for (int64_t i = (int64_t)u * blockDim.x + tid; i < zero16; i += (int64_t)gridDim.x * blockDim.x)
+    zero[i] = make_uint4(0, 0, 0, 0);
   const int nh = heads ? hsel : H;
   const int N = HS * geo.QB;
   const int n = geo.seq(u), tq0 = geo.t0(u);
@@ -672,7 +677,8 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
                             int* status, uint32_t* hist, cudaStream_t st, const int32_t* gidx,
-                            const int32_t* glen, const WaitProbe* test_probe) {
+                            const int32_t* glen, const WaitProbe* test_probe,
+                            size_t hist_zero_bytes) {
   const bool gather = gidx != nullptr;
   WaitProbe probe;
   probe.wait_cycles = kWaitCycles;
@@ -691,11 +697,13 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
   float* wg = reinterpret_cast<float*>(c);
   c += align256((size_t)units * p.N * 4);
   int32_t* tile_off = reinterpret_cast<int32_t*>(c);
-  if (p.QB > 1 || gather) hist = nullptr;
+  uint4* zero = reinterpret_cast<uint4*>(hist);   // zeroed by the prep kernel in every form
+  if (p.QB > 1 || gather) hist = nullptr;         // built by the epilogue in decode form only
 
   cudaError_t e = launch_pdl(score_tc_prep_kernel, dim3(units), dim3(1024), 0, st, q, w, heads,
                              hsel, H, p.HS, geo, pos, units, L, glen, (int)out_stride, qg, wg,
-                             tile_off, status);
+                             tile_off, status, zero,
+                             zero ? (int64_t)(hist_zero_bytes / 16) : (int64_t)0);
   if (e != cudaSuccess) return e;
   CUtensorMap tk, tq;   // (the gather copies key rows with cp.async: tk goes unused)
   if (!make_map(&tk, k, (uint64_t)nseq * L, (uint32_t)kTileKeys) ||

@@ -613,6 +613,33 @@ __global__ void __launch_bounds__(kSelThreads, 1) topk_group_kernel(
   }
 }
 
+// The score histogram of rows the scorer did not histogram (rows of several queries per
+// sequence): grid (chunks of kScatterChunk scores, rows); each CTA counts its chunk's keys
+// in shared memory and adds the occupied bins to the row's histogram (zeroed beforehand).
+__global__ void __launch_bounds__(kSelThreads) topk_build_hist_kernel(
+    const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
+    uint32_t* __restrict__ hist) {
+  pdl_prologue();
+  __shared__ uint32_t sh[kScoreHistBins];
+  const int t = threadIdx.x;
+  const int64_t row = blockIdx.y;
+  const int n = prefix_len(pos, row, L, nullptr);
+  const int start = blockIdx.x * kScatterChunk;
+  if (start >= n) return;
+  for (int b = t; b < kScoreHistBins; b += kSelThreads) sh[b] = 0;
+  __syncthreads();
+  const float* x = scores + row * stride;
+#pragma unroll
+  for (int j = 0; j < kScatterPer; ++j) {
+    const int e = start + j * kSelThreads + t;
+    if (e < n) atomicAdd(&sh[score_key(x[e]) >> (32 - kScoreHistBits)], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = hist + row * kScoreHistBins;
+  for (int b = t; b < kScoreHistBins; b += kSelThreads)
+    if (sh[b]) atomicAdd(gh + b, sh[b]);
+}
+
 // Exact selection for the rows topk_group_kernel leaves out (same overflow test, k > 4096).
 __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
     const float* __restrict__ scores, int64_t stride, const int32_t* __restrict__ pos, int64_t L,
@@ -862,16 +889,29 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     __syncthreads();
   }
   const bool fits = C <= (uint32_t)CAP;
-  // Candidates go to cin[0 .. C); the sort uses cscr as scratch.  The one-pass compaction:
-  // warp w takes the row's 32-key steps w, w + kWarps, ... (an even sample of the row) and
-  // appends its candidates to its own region of CAP / kWarps slots of cand; the regions are
-  // then packed into the (dead) key space.  A region that overflows sends the row through
-  // the two-pass compaction (count per warp slice, block scan, ballot ranks).
-  uint64_t* cin = cand;
-  uint64_t* cscr = sorted;
-  bool packed = false;
+  const uint64_t* res = sorted;   // the sorted pairs, for the output loop at the end
   if (fits) {
+    // The candidates are counted into sub-buckets while they are compacted -- bins
+    // [cut, btop], each split into 2^sb sub-buckets on the key bits below the bin, sb as
+    // large as kSubBuckets allows, numbered so that larger keys get smaller buckets -- then
+    // one scan, one scatter into bucket order and a rank inside each bucket (a pair counts
+    // the larger pairs of its bucket, mostly none) give every pair its output position,
+    // which is written to idx / vals directly.
+    const uint32_t nbins = btop - cut + 1;
+    int sb = 0;
+    while (sb < 20 && (nbins << (sb + 1)) <= (uint32_t)kSubBuckets) ++sb;
+    auto bucket_of = [&](uint32_t key) -> uint32_t {   // key >= kcut, so its bin >= cut
+      const uint32_t low = sb ? (key >> (32 - kScoreHistBits - sb)) & ((1u << sb) - 1u) : 0u;
+      const uint32_t bin = min(key >> (32 - kScoreHistBits), btop);   // (a given histogram
+      return ((btop - bin) << sb) | ((1u << sb) - 1u - low);           //  that disagrees)
+    };
+    uint32_t* sub = hist;   // the histogram is not read again on this path
     constexpr uint32_t kReg = (uint32_t)CAP / kWarps;
+    for (uint32_t b = t; b < (uint32_t)kSubBuckets; b += NT) sub[bpad(b)] = 0;
+    __syncthreads();
+    // one-pass compaction: warp w takes the row's 32-key steps w, w + kWarps, ... (an even
+    // sample of the row) and appends its candidates to its own region of CAP / kWarps
+    // slots of cand; every candidate is counted, stored or not
     uint32_t wc = 0;
 #pragma unroll 4
     for (int e0 = warp * 32; e0 < n; e0 += 32 * kWarps) {
@@ -880,49 +920,110 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       const bool take = e < n && key >= kcut;
       const uint32_t m = __ballot_sync(0xffffffffu, take);
       const uint32_t r = wc + __popc(m & below);
-      if (take && r < kReg) cand[warp * kReg + r] = compose(key, e);
+      if (take) {
+        atomicAdd(&sub[bpad(bucket_of(key))], 1u);
+        if (r < kReg) cand[warp * kReg + r] = compose(key, e);
+      }
       wc += __popc(m);
     }
-    if (lane == 0) warp_sums[warp] = wc;
-    if (!__syncthreads_or(wc > kReg ? 1 : 0)) {
-      uint32_t pre = 0, tot = 0;
-#pragma unroll
-      for (int w2 = 0; w2 < kWarps; ++w2) {
-        const uint32_t x = warp_sums[w2];
-        if (w2 < warp) pre += x;
-        tot += x;
+    const bool regions = !__syncthreads_or(wc > kReg ? 1 : 0);
+    if (!regions) {
+      // a region overflowed: the two-pass compaction (count per warp slice, block scan,
+      // ballot ranks) into cand[0 .. C)
+      if ((select && !given) || refined) {   // count this lane's candidates (else counted above)
+        cnt = 0;
+#pragma unroll 4
+        for (int e = w0 + lane; e < w1; e += 32) cnt += keys[e] >= kcut ? 1u : 0u;
       }
-      for (uint32_t i = lane; i < wc; i += 32) sorted[pre + i] = cand[warp * kReg + i];
-      C = tot;
-      cin = sorted;
-      cscr = cand;
-      packed = true;
-    }
-    __syncthreads();   // warp_sums is reused below
-  }
-  if (fits && !packed) {
-    if ((select && !given) || refined) {   // count this lane's candidates (else counted above)
-      cnt = 0;
-#pragma unroll 4
-      for (int e = w0 + lane; e < w1; e += 32) cnt += keys[e] >= kcut ? 1u : 0u;
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    uint32_t tot;
-    uint32_t p = __shfl_sync(0xffffffffu,
-                             block_excl_scan_nt<NT>(lane == 0 ? cnt : 0u, warp_sums, tot), 0);
-    C = min(tot, (uint32_t)CAP);
+      for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      uint32_t tot;
+      uint32_t p = __shfl_sync(0xffffffffu,
+                               block_excl_scan_nt<NT>(lane == 0 ? cnt : 0u, warp_sums, tot), 0);
+      C = min(tot, (uint32_t)CAP);
 #pragma unroll 4
-    for (int e0 = w0; e0 < w1; e0 += 32) {
-      const int e = e0 + lane;
-      const uint32_t key = e < w1 ? keys[e] : 0u;
-      const bool take = e < w1 && key >= kcut;
-      const uint32_t m = __ballot_sync(0xffffffffu, take);
-      const uint32_t r = p + __popc(m & below);
-      if (take && r < (uint32_t)CAP) cand[r] = compose(key, e);   // (a histogram that
-      p += __popc(m);                                            //  disagrees cannot overflow)
+      for (int e0 = w0; e0 < w1; e0 += 32) {
+        const int e = e0 + lane;
+        const uint32_t key = e < w1 ? keys[e] : 0u;
+        const bool take = e < w1 && key >= kcut;
+        const uint32_t m = __ballot_sync(0xffffffffu, take);
+        const uint32_t r = p + __popc(m & below);
+        if (take && r < (uint32_t)CAP) cand[r] = compose(key, e);   // (a histogram that
+        p += __popc(m);                                            //  disagrees cannot overflow)
+      }
     }
-  } else if (!fits) {
+    // exclusive scan of the bucket counts (thread t owns a run of kSubBuckets / NT buckets);
+    // the total is the number of candidates
+    constexpr int kPer = kSubBuckets / NT;
+    uint32_t c[kPer], local = 0, big = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      c[i] = sub[bpad(t * kPer + i)];
+      local += c[i];
+      big |= c[i] > kMaxBucket ? 1u : 0u;
+    }
+    uint32_t tot;
+    uint32_t run = block_excl_scan_nt<NT>(local, warp_sums, tot);
+    const bool crowded = __syncthreads_or(big ? 1 : 0);
+    if (regions) C = tot;
+    if (!crowded && tot == C) {
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        sub[bpad(t * kPer + i)] = run;   // bucket start, advanced to its end by the scatter
+        run += c[i];
+      }
+      __syncthreads();
+      // scatter into bucket order (the key space is dead: `sorted` takes the pairs)
+      if (regions) {
+        for (uint32_t i = lane; i < wc; i += 32) {
+          const uint64_t v = cand[warp * kReg + i];
+          sorted[atomicAdd(&sub[bpad(bucket_of((uint32_t)(v >> 32)))], 1u)] = v;
+        }
+      } else {
+        for (uint32_t i = t; i < C; i += NT) {
+          const uint64_t v = cand[i];
+          sorted[atomicAdd(&sub[bpad(bucket_of((uint32_t)(v >> 32)))], 1u)] = v;
+        }
+      }
+      __syncthreads();
+      // rank inside the bucket -> output position; bucket b spans [end(b - 1), end(b))
+      for (uint32_t i = t; i < C; i += NT) {
+        const uint64_t v = sorted[i];
+        const uint32_t b = bucket_of((uint32_t)(v >> 32));
+        const uint32_t s0 = b ? sub[bpad(b - 1)] : 0u, s1 = sub[bpad(b)];
+        uint32_t r = 0;
+        for (uint32_t j = s0; j < s1; ++j) r += sorted[j] > v ? 1u : 0u;
+        const uint32_t o = s0 + r;
+        if (o < target) {
+          const int32_t e = (int32_t)(~(uint32_t)(v & 0xffffffffu));   // position in the row
+          idx[row * topk + o] = imap ? imap[e] : e;
+          if (vals) vals[row * topk + o] = key_score((uint32_t)(v >> 32));
+        }
+      }
+      for (int i = (int)target + t; i < topk; i += NT) {
+        idx[row * topk + i] = -1;
+        if (vals) vals[row * topk + i] = __int_as_float(0xff800000);
+      }
+      return;
+    }
+    // crowded buckets (many equal keys), or a count that disagrees with the compaction:
+    // bitonic sort of the candidates instead
+    if (regions) {
+      if (lane == 0) warp_sums[warp] = wc;
+      __syncthreads();
+      uint32_t pre = 0;
+      for (int w2 = 0; w2 < warp; ++w2) pre += warp_sums[w2];
+      for (uint32_t i = lane; i < wc && pre + i < (uint32_t)CAP; i += 32)
+        sorted[pre + i] = cand[warp * kReg + i];
+    } else {
+      for (uint32_t i = t; i < C; i += NT) sorted[i] = cand[i];
+    }
+    int sortn = NT;
+    while ((uint32_t)sortn < C) sortn <<= 1;
+    for (int i = (int)C + t; i < sortn; i += NT) sorted[i] = 0ull;
+    __syncthreads();
+    row_bitonic<NT, RC::kEMax>(sorted, sortn);
+  } else {
     // crowded cutoff bin: exact threshold by a radix select over the resident keys, then
     // exactly `target` pairs (above the threshold, then equal ones in index order)
     uint32_t prefix = 0, mask = 0, kneed = target;
@@ -1004,24 +1105,19 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     if (t == 0) { red[0] = 0xffffffffu; red[1] = 0; }
     __syncthreads();
     block_minmax<NT>(lo_dummy, btop, red);
-  }
-  __syncthreads();
-  // keys are dead from here on: their space is the sort's scratch.  The per-bin counts of
-  // the candidates are the histogram's when every key of bins [cut, btop] is a candidate.
-  const uint32_t* bin_counts = (select && fits && !refined) ? hist : nullptr;
-  const uint64_t* res = cin;   // the counting sort leaves its result in place
-  if (C > 0 && !group_sort_adaptive<NT>(cin, C, cscr, hist,
-                               reinterpret_cast<uint8_t*>(rbuf) + RC::kAuxOff, cut, btop,
-                               warp_sums, s_flag, s_nsub, bin_counts)) {
-    res = sorted;
-    int sortn = NT;
-    while ((uint32_t)sortn < C) sortn <<= 1;
-    if (cin == cand)
-      for (int i = t; i < sortn; i += NT) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
-    else
-      for (int i = (int)C + t; i < sortn; i += NT) sorted[i] = 0ull;
     __syncthreads();
-    row_bitonic<NT, RC::kEMax>(sorted, sortn);
+    // keys are dead from here on: their space is the sort's scratch
+    res = cand;   // the counting sort leaves its result in place
+    if (!group_sort_adaptive<NT>(cand, C, sorted, hist,
+                                 reinterpret_cast<uint8_t*>(rbuf) + RC::kAuxOff, cut, btop,
+                                 warp_sums, s_flag, s_nsub, nullptr)) {
+      res = sorted;
+      int sortn = NT;
+      while ((uint32_t)sortn < C) sortn <<= 1;
+      for (int i = t; i < sortn; i += NT) sorted[i] = (uint32_t)i < C ? cand[i] : 0ull;
+      __syncthreads();
+      row_bitonic<NT, RC::kEMax>(sorted, sortn);
+    }
   }
   // outputs, four per thread per step so that the index-map loads overlap
   for (int i0 = t; i0 < topk; i0 += 4 * NT) {
@@ -1103,6 +1199,17 @@ cudaError_t launch_topk_hist(const float* scores, int64_t stride, const int32_t*
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_hist_overflow_kernel, dim3(rows), dim3(kThreads), ov_smem, st, scores,
                     stride, pos, L, hist, topk, sortn, idx, vals);
+}
+
+cudaError_t launch_build_hist(const float* scores, int64_t stride, const int32_t* pos, int64_t L,
+                              int rows, uint32_t* hist, cudaStream_t st) {
+  const dim3 grid((unsigned)((L + kScatterChunk - 1) / kScatterChunk), (unsigned)rows);
+  return launch_pdl(topk_build_hist_kernel, grid, dim3(kSelThreads), 0, st, scores, stride, pos, L,
+                    hist);
+}
+
+size_t topk_hist_zero_bytes(int64_t rows) {
+  return align256((size_t)rows * kScoreHistBins * 4) + align256((size_t)rows * kMaxGroups * 4);
 }
 
 size_t topk_hist_ws_bytes(int64_t rows, int topk) {

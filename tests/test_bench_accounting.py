@@ -49,5 +49,7 @@ def test_forms_and_launch_counts():
     assert bench.misa_step_launches(WORKLOADS["dsv32_decode_32k"]) == 5
     # 128K decode rows exceed the row top-k's 40960: scatter + group
     assert bench.misa_step_launches(WORKLOADS["glm5_decode_128k"]) == 6
+    # 4 queries per sequence over 32K: histogram pass + row top-k
+    assert bench.misa_step_launches(WORKLOADS["dsv32_mtp_32k"]) == 6
     # prefill: three tensor-core router kernels (hi/lo split, partial blocks, GEMM + top-h)
     assert bench.misa_step_launches(WORKLOADS["dsv32_prefill_16k"]) == 7

@@ -436,15 +436,26 @@ def measure_workload(M, wl, args, dev, world, rank, peaks, headline: bool):
     recalls = {"misa": recall(idx, didx), "misa_dagger": recall(gidx, didx)}
     if hisa_on:
         recalls["hisa_block_filter"] = recall(hidx, didx)
-    # the routed scoring kernel alone (misa_score_rows: the scorer of misa_score_topk with the
-    # same launch configuration), on the heads the MISA steps routed
+    # the routed scoring kernel alone (the scorer of misa_score_topk with the same launch
+    # configuration), on the heads the MISA steps routed: CUDA events around that kernel's
+    # launch, inside the library (the gather kernel before it is left out), averaged over
+    # the steps; and the whole misa_score_rows call (gather + scoring kernel) for reference
     score_buf = torch.empty((nseq, T, wl.L), dtype=torch.float32, device=dev)
 
     def score_step(i):
         q, w, k, pos = sets[i % 2]
         M.misa_score_rows(q, w, k, heads, pos, scores=score_buf)
 
-    ms_score_kernel = timed(score_step, args.steps, args.warmup)
+    ms_score_call = timed(score_step, args.steps, args.warmup)
+
+    def score_kernel(i):
+        q, w, k, pos = sets[i % 2]
+        return M.misa_testing_score_rows_timed(q, w, k, heads, pos, scores=score_buf)
+
+    for i in range(args.warmup):
+        score_kernel(i)
+    kernel_ms = [score_kernel(i) for i in range(args.steps)]
+    ms_score_kernel = sum(kernel_ms) / len(kernel_ms)
     del score_buf
     M.misa_check_device_status(dev)
 
@@ -461,7 +472,8 @@ def measure_workload(M, wl, args, dev, world, rank, peaks, headline: bool):
         "paths": {
             "misa": {"value": units * world / (ms_misa * 1e-3), "ms_per_step": ms_misa,
                      "ms_pool": call_ms[0], "ms_route": call_ms[1], "ms_score_topk": call_ms[2],
-                     "ms_score_kernel_alone": ms_score_kernel},
+                     "ms_score_kernel_alone": ms_score_kernel,
+                     "ms_score_rows_call": ms_score_call},
             "dsa": {"value": units * world / (ms_dsa * 1e-3), "ms_per_step": ms_dsa},
             "misa_dagger": {"value": units * world / (ms_dagger * 1e-3),
                             "ms_per_step": ms_dagger},

@@ -1,15 +1,17 @@
 /*
  * misa_testing.h -- test-only entry points of the B200 MISA indexer library.
  *
- * These are not part of the indexer's API (include/misa.h).  They exist so that a
- * test can reach two code paths the ordinary entry points only take in rare
- * conditions, and compare them with an independent CPU reference:
+ * These are not part of the indexer's API (include/misa.h).  Two of them exist so that a
+ * test can reach code paths the ordinary entry points only take in rare conditions,
+ * and compare them with an independent CPU reference:
  *   - the CUDA-core scorer, which misa_score_topk / dsa_score_topk / the MISA-dagger
  *     re-rank fall back to when the tensor-core scorer cannot take a shape (nseq * L
  *     at or above 2^31, or no driver entry point for tensor maps);
  *   - the expiry path of the tensor-core scorer's bounded waits: record
  *     MISA_ERR_DEVICE_TIMEOUT, let the copies and MMAs already in flight finish,
  *     free the tensor memory, and return, leaving the context usable.
+ * The third times the tensor-core scoring kernel on its own, for the roofline of the
+ * benchmark.
  * Conventions (pointers, layouts, ownership, workspace, status codes) are those of
  * include/misa.h.
  */
@@ -54,6 +56,20 @@ int misa_testing_score_rows_wait_expiry(const uint16_t* q, const float* w, const
                                         int T, int H, int d, int64_t L, int h, float* scores,
                                         void* ws, size_t ws_bytes, long long wait_cycles,
                                         int skip_tile, void* stream);
+
+/*
+ * misa_score_rows on the tensor-core scorer, and the device time of its scoring kernel
+ * alone: two CUDA events recorded on `stream` around that kernel's launch (after the
+ * gather kernel that precedes it, which they leave out).  Blocks until the kernel has
+ * finished, then writes the elapsed milliseconds to *kernel_ms (host memory).  Returns
+ * MISA_ERR_UNSUPPORTED where misa_score_rows would not use the tensor-core scorer,
+ * MISA_ERR_INVALID_ARG when kernel_ms is NULL.  Workspace: misa_workspace_size(
+ * MISA_OP_SCORE_ROWS, ...).
+ */
+int misa_testing_score_rows_timed(const uint16_t* q, const float* w, const uint16_t* k,
+                                  const int32_t* heads, const int32_t* pos, int nseq, int T,
+                                  int H, int d, int64_t L, int h, float* scores, void* ws,
+                                  size_t ws_bytes, float* kernel_ms, void* stream);
 
 #ifdef __cplusplus
 }

@@ -28,6 +28,7 @@ from ._binding import (  # noqa: F401
     misa_score_topk,
     misa_score_topk_noalloc,
     misa_testing_score_rows_wait_expiry,
+    misa_testing_score_rows_timed,
     misa_testing_score_simt,
     misa_workspace_size,
     workspace,

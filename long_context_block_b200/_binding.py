@@ -56,6 +56,9 @@ _SIGS = {
     "misa_testing_score_rows_wait_expiry": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int,
                                                      _c_int, _c_i64, _c_int, _p, _p, _c_sz,
                                                      ctypes.c_longlong, _c_int, _p]),
+    "misa_testing_score_rows_timed": (_c_int, [_p, _p, _p, _p, _p, _c_int, _c_int, _c_int,
+                                               _c_int, _c_i64, _c_int, _p, _p, _c_sz,
+                                               ctypes.POINTER(ctypes.c_float), _p]),
     "misa_status_string": (ctypes.c_char_p, [_c_int]),
     "misa_check_device_status": (_c_int, [_p, _p]),
 }
@@ -421,3 +424,28 @@ def misa_testing_score_rows_wait_expiry(q, w, k, heads, pos, wait_cycles: int, s
                                                     _ptr(scores), _ptr(ws), ws.numel(),
                                                     int(wait_cycles), int(skip_tile), _stream()))
     return scores
+
+
+def misa_testing_score_rows_timed(q, w, k, heads, pos, scores: torch.Tensor | None = None):
+    """misa_score_rows on the tensor-core scorer; returns the device milliseconds of its
+    scoring kernel alone (CUDA events around that launch; the call waits for it)."""
+    q, k = _bits(q, "q"), _bits(k, "k")
+    w = _dev(w, "w", torch.float32)
+    pos = _dev(pos, "pos", torch.int32)
+    nseq, T, H, d = q.shape
+    L = k.shape[1]
+    if heads is not None:
+        heads = _dev(heads, "heads", torch.int32)
+    h = heads.shape[-1] if heads is not None else H
+    if scores is None:
+        scores = torch.empty((nseq, T, L), dtype=torch.float32, device=q.device)
+    nb = misa_workspace_size(OP_SCORE_ROWS, nseq, T, H, d, L, 1, h, 1, 1)
+    if nb == 0:
+        raise MisaError("misa_workspace_size", 1)
+    ws = _WS.get(nb, q.device)
+    ms = ctypes.c_float(0.0)
+    _check("misa_testing_score_rows_timed",
+           _lib.misa_testing_score_rows_timed(_ptr(q), _ptr(w), _ptr(k), _ptr(heads), _ptr(pos),
+                                              nseq, T, H, d, L, h, _ptr(scores), _ptr(ws),
+                                              ws.numel(), ctypes.byref(ms), _stream()))
+    return float(ms.value)

@@ -389,4 +389,36 @@ int misa_testing_score_rows_wait_expiry(const uint16_t* q, const float* w, const
                                      (cudaStream_t)stream, nullptr, nullptr, &probe));
 }
 
+int misa_testing_score_rows_timed(const uint16_t* q, const float* w, const uint16_t* k,
+                                  const int32_t* heads, const int32_t* pos, int nseq, int T,
+                                  int H, int d, int64_t L, int h, float* scores, void* ws,
+                                  size_t ws_bytes, float* kernel_ms, void* stream) {
+  MISA_TRY(check_shape(nseq, T, H, d, L));
+  if (h < 1 || h > H || kernel_ms == nullptr) return MISA_ERR_INVALID_ARG;
+  if (heads && h > MISA_MAX_ROUTED) return MISA_ERR_UNSUPPORTED;
+  const int nh = heads ? h : H;
+  if (!score_tc_supported(nseq, T, nh, L)) return MISA_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)nseq * T;
+  MISA_TRY(check_dev(q, rows * H * d * 2, 16));
+  MISA_TRY(check_dev(w, rows * H * 4, 4));
+  MISA_TRY(check_dev(k, (size_t)nseq * L * d * 2, 16));
+  MISA_TRY(check_dev(pos, rows * 4, 4));
+  if (heads) MISA_TRY(check_dev(heads, rows * h * 4, 4));
+  MISA_TRY(check_dev(scores, rows * L * 4, 4));
+  MISA_TRY(check_ws(ws, ws_bytes, kStatusBytes + score_tc_ws_bytes(nseq, T, nh)));
+  KernelTimer timer;
+  MISA_TRY(cuda_status(cudaEventCreate(&timer.begin)));
+  cudaError_t e = cudaEventCreate(&timer.end);
+  if (e == cudaSuccess) {
+    e = launch_score_tc(q, w, k, heads, h, pos, nseq, T, H, L, scores, L, ws_region(ws, 0),
+                        status_word(ws), nullptr, (cudaStream_t)stream, nullptr, nullptr,
+                        nullptr, 0, &timer);
+    if (e == cudaSuccess) e = cudaEventSynchronize(timer.end);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(kernel_ms, timer.begin, timer.end);
+    cudaEventDestroy(timer.end);
+  }
+  cudaEventDestroy(timer.begin);
+  return cuda_status(e);
+}
+
 }  // extern "C"

@@ -121,6 +121,12 @@ struct WaitProbe {
   long long wait_cycles;
   int skip_tile;
 };
+//   timer (nullable; benchmark only): events recorded on st directly before and after the
+//   scoring kernel's launch (after the prep kernel).
+struct KernelTimer {
+  cudaEvent_t begin;
+  cudaEvent_t end;
+};
 cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k,
                             const int32_t* heads, int hsel, const int32_t* pos, int nseq, int T,
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
@@ -128,7 +134,7 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
                             const int32_t* gather_ids = nullptr,
                             const int32_t* gather_len = nullptr,
                             const WaitProbe* test_probe = nullptr,
-                            size_t hist_zero_bytes = 0);
+                            size_t hist_zero_bytes = 0, const KernelTimer* timer = nullptr);
 
 // K5 -- per-row top-k selection (topk.cu).
 //   Row r has len = gather_len ? gather_len[r] : pos[r] + 1 scores at scores + r * stride.

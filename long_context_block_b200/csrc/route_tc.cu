@@ -340,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
       float dot = 0.f;
       if (ok && !warp_wait(&full[s], (it / kStages) & 1, abort_flag, status)) ok = false;
       if (ok && M > mfull) {
+        float d4[4] = {0.f, 0.f, 0.f, 0.f};   // four chains, so the FMAs overlap
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const uint8_t* arow = base + kStageBase + s * kATileBytes + hf * kAHalf + r * 128;
@@ -349,12 +350,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
           for (int c = 0; c < 8; ++c) {   // 16-byte chunk c of the row (128-byte swizzle)
             const uint4 x = *reinterpret_cast<const uint4*>(arow + ((c ^ (r & 7)) << 4));
             const float4 a = kv[2 * c], b = kv[2 * c + 1];
-            dot = fmaf(bf16lo(x.x), a.x, dot); dot = fmaf(bf16hi(x.x), a.y, dot);
-            dot = fmaf(bf16lo(x.y), a.z, dot); dot = fmaf(bf16hi(x.y), a.w, dot);
-            dot = fmaf(bf16lo(x.z), b.x, dot); dot = fmaf(bf16hi(x.z), b.y, dot);
-            dot = fmaf(bf16lo(x.w), b.z, dot); dot = fmaf(bf16hi(x.w), b.w, dot);
+            d4[0] = fmaf(bf16lo(x.x), a.x, d4[0]); d4[1] = fmaf(bf16hi(x.x), a.y, d4[1]);
+            d4[2] = fmaf(bf16lo(x.y), a.z, d4[2]); d4[3] = fmaf(bf16hi(x.y), a.w, d4[3]);
+            d4[0] = fmaf(bf16lo(x.z), b.x, d4[0]); d4[1] = fmaf(bf16hi(x.z), b.y, d4[1]);
+            d4[2] = fmaf(bf16lo(x.w), b.z, d4[2]); d4[3] = fmaf(bf16hi(x.w), b.w, d4[3]);
           }
         }
+        dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
       }
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(&empty[s]);   // this warp is done with the stage
@@ -378,18 +380,20 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                                    (uint32_t)(acc * kItemBlocks);
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};   // four chains, so the adds overlap
             for (int c0 = 0; c0 < mwarp; c0 += 32) {
               float v[32];
               tmem_ld32(taddr + c0, v);
               if (c0 + 32 <= mrow) {
 #pragma unroll
-                for (int cc = 0; cc < 32; ++cc) sum += fmaxf(v[cc], 0.f);
+                for (int cc = 0; cc < 32; ++cc) s4[cc & 3] += fmaxf(v[cc], 0.f);
               } else {
 #pragma unroll
                 for (int cc = 0; cc < 32; ++cc)
-                  if (c0 + cc < mrow) sum += fmaxf(v[cc], 0.f);
+                  if (c0 + cc < mrow) s4[cc & 3] += fmaxf(v[cc], 0.f);
               }
             }
+            sum += (s4[0] + s4[1]) + (s4[2] + s4[3]);
             tc_fence_before();
             mbar_arrive(&accempty[acc]);
           }

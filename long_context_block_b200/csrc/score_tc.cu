@@ -542,9 +542,18 @@ __global__ void __launch_bounds__(1024) score_tc_prep_kernel(
         int Pmax = 0;
         if (glen)   // gather mode: one row per unit, its token-list length
           Pmax = min(max(glen[uu], 0), gmax);
-        else
-          for (int qq = 0; qq < geo.QB && ta + qq < geo.T; ++qq)
-            Pmax = max(Pmax, prefix_len(pos, (int64_t)nn * geo.T + ta + qq, L, status));
+        else   // eight independent loads per step
+          for (int q0 = 0; q0 < geo.QB && ta + q0 < geo.T; q0 += 8) {
+            int p8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int qq = q0 + j;
+              p8[j] = (qq < geo.QB && ta + qq < geo.T)
+                          ? prefix_len(pos, (int64_t)nn * geo.T + ta + qq, L, status) : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) Pmax = max(Pmax, p8[j]);
+          }
         v = (Pmax + kTileKeys - 1) / kTileKeys;
       }
       int incl = v;
@@ -614,7 +623,7 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
                        const int32_t* pos, const int32_t* tile_off, int units, Units geo,
                        int64_t L, float* out, int64_t out_stride, int* status, uint32_t* hist,
                        const int32_t* gidx, const int32_t* glen, const uint16_t* kraw,
-                       const WaitProbe& probe, cudaStream_t st) {
+                       const WaitProbe& probe, const KernelTimer* timer, cudaStream_t st) {
   using C = Cfg<HS, QB>;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<HS, QB, kGather>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -622,9 +631,12 @@ cudaError_t launch_cfg(const CUtensorMap& tk, const CUtensorMap& tq, const float
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return launch_pdl(score_tc_kernel<HS, QB, kGather>, dim3(sms), dim3(C::kThreads),
-                    (size_t)C::kSmemBytes, st, tk, tq, wg, pos, tile_off, units, geo, L, out,
-                    out_stride, status, hist, gidx, glen, kraw, probe);
+  if (timer && (e = cudaEventRecord(timer->begin, st)) != cudaSuccess) return e;
+  e = launch_pdl(score_tc_kernel<HS, QB, kGather>, dim3(sms), dim3(C::kThreads),
+                 (size_t)C::kSmemBytes, st, tk, tq, wg, pos, tile_off, units, geo, L, out,
+                 out_stride, status, hist, gidx, glen, kraw, probe);
+  if (e == cudaSuccess && timer) e = cudaEventRecord(timer->end, st);
+  return e;
 }
 
 // Shape of the work units for nh heads and T queries per sequence.
@@ -678,7 +690,7 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
                             int H, int64_t L, float* out, int64_t out_stride, void* scratch,
                             int* status, uint32_t* hist, cudaStream_t st, const int32_t* gidx,
                             const int32_t* glen, const WaitProbe* test_probe,
-                            size_t hist_zero_bytes) {
+                            size_t hist_zero_bytes, const KernelTimer* timer) {
   const bool gather = gidx != nullptr;
   WaitProbe probe;
   probe.wait_cycles = kWaitCycles;
@@ -712,11 +724,11 @@ cudaError_t launch_score_tc(const uint16_t* q, const float* w, const uint16_t* k
 #define MISA_TC_CASE(HS_, QB_)                                                                  \
   if (p.HS == HS_ && p.QB == QB_)                                                               \
     return launch_cfg<HS_, QB_, false>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride, \
-                                       status, hist, nullptr, nullptr, k, probe, st);
+                                       status, hist, nullptr, nullptr, k, probe, timer, st);
 #define MISA_TC_GATHER_CASE(HS_)                                                                \
   if (p.HS == HS_)                                                                              \
     return launch_cfg<HS_, 1, true>(tk, tq, wg, pos, tile_off, units, geo, L, out, out_stride,    \
-                                    status, nullptr, gidx, glen, k, probe, st);
+                                    status, nullptr, gidx, glen, k, probe, timer, st);
   if (gather) {
     MISA_TC_GATHER_CASE(16)
     MISA_TC_GATHER_CASE(32)

@@ -741,7 +741,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   __shared__ __align__(16) uint32_t hist[kSubBucketWords];     // histogram, then buckets
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t red[2];
-  __shared__ uint32_t s_cut, s_total, s_big, s_flag, s_digit, s_above, s_top, s_nsub;
+  __shared__ uint32_t s_cut, s_total, s_big, s_flag, s_digit, s_above, s_top, s_nsub, s_spill;
   __shared__ __align__(8) uint64_t lbar;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t row = row0 + blockIdx.x;
@@ -827,10 +827,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
   // selected) or this warp's candidate count (cutoff given)
   const uint32_t kgiven = cut << (32 - kScoreHistBits);
   uint32_t lo = 0xffffffffu, hi = 0, cnt = 0;
-#pragma unroll 4
-  for (int e = w0 + lane; e < w1; e += 32) {
-    const uint32_t kk = score_key(__uint_as_float(keys[e]));
-    keys[e] = kk;
+  auto note = [&](uint32_t kk) {
     const uint32_t b = kk >> (32 - kScoreHistBits);
     if (!select) {
       lo = min(lo, b);
@@ -839,6 +836,36 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       cnt += kk >= kgiven ? 1u : 0u;
     } else {
       atomicAdd(&hist[b], 1u);
+    }
+  };
+  if (hb == 0) {   // the keys start 16-byte aligned: lane l takes keys e .. e + 3, e = w0 + 4 l + 128 i
+#pragma unroll 2
+    for (int e = w0 + 4 * lane; e < w1; e += 128) {
+      if (e + 4 <= w1) {
+        uint4 v = *reinterpret_cast<const uint4*>(keys + e);
+        v.x = score_key(__uint_as_float(v.x));
+        v.y = score_key(__uint_as_float(v.y));
+        v.z = score_key(__uint_as_float(v.z));
+        v.w = score_key(__uint_as_float(v.w));
+        *reinterpret_cast<uint4*>(keys + e) = v;
+        note(v.x);
+        note(v.y);
+        note(v.z);
+        note(v.w);
+      } else {
+        for (int u = e; u < w1; ++u) {
+          const uint32_t kk = score_key(__uint_as_float(keys[u]));
+          keys[u] = kk;
+          note(kk);
+        }
+      }
+    }
+  } else {
+#pragma unroll 4
+    for (int e = w0 + lane; e < w1; e += 32) {
+      const uint32_t kk = score_key(__uint_as_float(keys[e]));
+      keys[e] = kk;
+      note(kk);
     }
   }
   __syncthreads();
@@ -906,27 +933,80 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       return ((btop - bin) << sb) | ((1u << sb) - 1u - low);           //  that disagrees)
     };
     uint32_t* sub = hist;   // the histogram is not read again on this path
-    constexpr uint32_t kReg = (uint32_t)CAP / kWarps;
+    // Candidate slots: a region of kReg per warp, then a shared pool of the rest of cand,
+    // then (when the key space holds CAP pairs past the row's keys and past the CAP pairs
+    // the scatter writes at its start) a spill area there.  A pair that finds no slot
+    // sends the row through the two-pass compaction.
+    constexpr uint32_t kReg = (uint32_t)CAP * 7u / 10u / kWarps;
+    constexpr uint32_t kPool = (uint32_t)CAP - kReg * kWarps;
+    uint64_t* pool = cand + kReg * kWarps;
+    const uint32_t kfree = (uint32_t)((hb + 4u * (uint32_t)n + 7u) / 8u);   // first free pair
+    const uint32_t spill_cap =
+        (hb == 0 && kfree >= (uint32_t)CAP && kfree + (uint32_t)CAP <= (uint32_t)RC::kKeyPairs)
+            ? (uint32_t)CAP : 0u;
+    uint64_t* spill = rbuf + kfree;
     for (uint32_t b = t; b < (uint32_t)kSubBuckets; b += NT) sub[bpad(b)] = 0;
+    if (t == 0) s_spill = 0;
     __syncthreads();
-    // one-pass compaction: warp w takes the row's 32-key steps w, w + kWarps, ... (an even
-    // sample of the row) and appends its candidates to its own region of CAP / kWarps
-    // slots of cand; every candidate is counted, stored or not
-    uint32_t wc = 0;
-#pragma unroll 4
-    for (int e0 = warp * 32; e0 < n; e0 += 32 * kWarps) {
-      const int e = e0 + lane;
-      const uint32_t key = e < n ? keys[e] : 0u;
-      const bool take = e < n && key >= kcut;
-      const uint32_t m = __ballot_sync(0xffffffffu, take);
-      const uint32_t r = wc + __popc(m & below);
-      if (take) {
-        atomicAdd(&sub[bpad(bucket_of(key))], 1u);
-        if (r < kReg) cand[warp * kReg + r] = compose(key, e);
+    // one-pass compaction: warp w takes the row's key steps w, w + kWarps, ... (an even
+    // sample of the row) and appends its candidates to its own region, then to the pool
+    // and the spill area; every candidate is counted in its sub-bucket, stored or not
+    auto put = [&](uint32_t r, uint32_t key, int ee) {
+      atomicAdd(&sub[bpad(bucket_of(key))], 1u);
+      if (r < kReg) {
+        cand[warp * kReg + r] = compose(key, ee);
+      } else {
+        const uint32_t p = atomicAdd(&s_spill, 1u);
+        if (p < kPool)
+          pool[p] = compose(key, ee);
+        else if (p - kPool < spill_cap)
+          spill[p - kPool] = compose(key, ee);
       }
-      wc += __popc(m);
+    };
+    uint32_t wc = 0;
+    if (hb == 0) {   // 128-key steps: lane l takes keys e .. e + 3
+#pragma unroll 2
+      for (int e0 = warp * 128; e0 < n; e0 += 128 * kWarps) {
+        const int e = e0 + 4 * lane;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (e + 4 <= n) {
+          v = *reinterpret_cast<const uint4*>(keys + e);
+        } else {
+          if (e < n) v.x = keys[e];
+          if (e + 1 < n) v.y = keys[e + 1];
+          if (e + 2 < n) v.z = keys[e + 2];
+        }
+        const bool t0 = e < n && v.x >= kcut, t1 = e + 1 < n && v.y >= kcut;
+        const bool t2 = e + 2 < n && v.z >= kcut, t3 = e + 3 < n && v.w >= kcut;
+        const uint32_t c = (uint32_t)t0 + (uint32_t)t1 + (uint32_t)t2 + (uint32_t)t3;
+        // lane prefix of the counts from ballots of their bits
+        const uint32_t b0 = __ballot_sync(0xffffffffu, c & 1u);
+        const uint32_t b1 = __ballot_sync(0xffffffffu, c & 2u);
+        const uint32_t b2 = __ballot_sync(0xffffffffu, c & 4u);
+        uint32_t r = wc + __popc(b0 & below) + 2u * __popc(b1 & below) + 4u * __popc(b2 & below);
+        if (t0) put(r++, v.x, e);
+        if (t1) put(r++, v.y, e + 1);
+        if (t2) put(r++, v.z, e + 2);
+        if (t3) put(r++, v.w, e + 3);
+        wc += __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
+      }
+    } else {   // 32-key steps
+#pragma unroll 4
+      for (int e0 = warp * 32; e0 < n; e0 += 32 * kWarps) {
+        const int e = e0 + lane;
+        const uint32_t key = e < n ? keys[e] : 0u;
+        const bool take = e < n && key >= kcut;
+        const uint32_t m = __ballot_sync(0xffffffffu, take);
+        if (take) put(wc + __popc(m & below), key, e);
+        wc += __popc(m);
+      }
     }
-    const bool regions = !__syncthreads_or(wc > kReg ? 1 : 0);
+    __syncthreads();
+    const uint32_t novf = s_spill;                    // pairs past the regions
+    const bool regions = novf <= kPool + spill_cap;
+    const uint32_t npool = regions ? min(novf, kPool) : 0u;
+    const uint32_t nspill = regions ? novf - npool : 0u;
+    const uint32_t wreg = min(wc, kReg);              // pairs in this warp's region
     if (!regions) {
       // a region overflowed: the two-pass compaction (count per warp slice, block scan,
       // ballot ranks) into cand[0 .. C)
@@ -975,8 +1055,12 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       __syncthreads();
       // scatter into bucket order (the key space is dead: `sorted` takes the pairs)
       if (regions) {
-        for (uint32_t i = lane; i < wc; i += 32) {
+        for (uint32_t i = lane; i < wreg; i += 32) {
           const uint64_t v = cand[warp * kReg + i];
+          sorted[atomicAdd(&sub[bpad(bucket_of((uint32_t)(v >> 32)))], 1u)] = v;
+        }
+        for (uint32_t i = t; i < npool + nspill; i += NT) {
+          const uint64_t v = i < npool ? pool[i] : spill[i - npool];
           sorted[atomicAdd(&sub[bpad(bucket_of((uint32_t)(v >> 32)))], 1u)] = v;
         }
       } else {
@@ -986,19 +1070,37 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
         }
       }
       __syncthreads();
-      // rank inside the bucket -> output position; bucket b spans [end(b - 1), end(b))
-      for (uint32_t i = t; i < C; i += NT) {
-        const uint64_t v = sorted[i];
-        const uint32_t b = bucket_of((uint32_t)(v >> 32));
-        const uint32_t s0 = b ? sub[bpad(b - 1)] : 0u, s1 = sub[bpad(b)];
-        uint32_t r = 0;
-        for (uint32_t j = s0; j < s1; ++j) r += sorted[j] > v ? 1u : 0u;
-        const uint32_t o = s0 + r;
-        if (o < target) {
-          const int32_t e = (int32_t)(~(uint32_t)(v & 0xffffffffu));   // position in the row
-          idx[row * topk + o] = imap ? imap[e] : e;
-          if (vals) vals[row * topk + o] = key_score((uint32_t)(v >> 32));
+      // rank inside the bucket -> output position; bucket b spans [end(b - 1), end(b)).
+      // Four pairs per thread per step, so that their shared-memory chains overlap.
+      for (uint32_t i0 = t; i0 < C; i0 += 4 * NT) {
+        uint64_t v[4];
+        uint32_t o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = i0 + u * NT < C ? sorted[i0 + u * NT] : 0ull;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          o[u] = 0xffffffffu;
+          if (i0 + u * NT < C) {
+            const uint32_t b = bucket_of((uint32_t)(v[u] >> 32));
+            const uint32_t s0 = b ? sub[bpad(b - 1)] : 0u, s1 = sub[bpad(b)];
+            uint32_t r = 0;
+            if (s1 - s0 > 1u)
+              for (uint32_t j = s0; j < s1; ++j) r += sorted[j] > v[u] ? 1u : 0u;
+            o[u] = s0 + r;
+          }
         }
+        int32_t id[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int32_t e = (int32_t)(~(uint32_t)(v[u] & 0xffffffffu));   // position in the row
+          id[u] = (imap && o[u] < target) ? imap[e] : e;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (o[u] < target) {
+            idx[row * topk + o[u]] = id[u];
+            if (vals) vals[row * topk + o[u]] = key_score((uint32_t)(v[u] >> 32));
+          }
       }
       for (int i = (int)target + t; i < topk; i += NT) {
         idx[row * topk + i] = -1;
@@ -1009,12 +1111,17 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     // crowded buckets (many equal keys), or a count that disagrees with the compaction:
     // bitonic sort of the candidates instead
     if (regions) {
-      if (lane == 0) warp_sums[warp] = wc;
+      if (lane == 0) warp_sums[warp] = wreg;
       __syncthreads();
-      uint32_t pre = 0;
-      for (int w2 = 0; w2 < warp; ++w2) pre += warp_sums[w2];
-      for (uint32_t i = lane; i < wc && pre + i < (uint32_t)CAP; i += 32)
+      uint32_t pre = 0, all = 0;
+      for (int w2 = 0; w2 < kWarps; ++w2) {
+        if (w2 < warp) pre += warp_sums[w2];
+        all += warp_sums[w2];
+      }
+      for (uint32_t i = lane; i < wreg && pre + i < (uint32_t)CAP; i += 32)
         sorted[pre + i] = cand[warp * kReg + i];
+      for (uint32_t i = t; i < npool + nspill && all + i < (uint32_t)CAP; i += NT)
+        sorted[all + i] = i < npool ? pool[i] : spill[i - npool];
     } else {
       for (uint32_t i = t; i < C; i += NT) sorted[i] = cand[i];
     }
@@ -1238,7 +1345,7 @@ cudaError_t launch_topk(const float* scores, int64_t stride, const int32_t* pos,
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (topk <= 3072 && rows >= 2 * sms)
-      return launch_row<256, 3072, kRowCap, 2>(scores, stride, pos, L, gather_len, index_map,
+      return launch_row<512, 3072, kRowCap, 2>(scores, stride, pos, L, gather_len, index_map,
                                                nullptr, rows, topk, idx, vals, status, st);
     if (rows >= sms)
       return launch_row<512, 8192, kRowCap, 1>(scores, stride, pos, L, gather_len, index_map,

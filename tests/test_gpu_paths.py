@@ -1,8 +1,9 @@
 """Code paths the ordinary entry points take only in rare conditions, against the fp64
 oracle (GPU): the CUDA-core scorer (the fallback of misa_score_topk / dsa_score_topk /
 the MISA-dagger re-rank), the expiry path of the tensor-core scorer's bounded waits,
-the h = H^I invariant (MISA page, Eq. 9 with every head routed is Eq. 1), and the
-host-side rejection of a too-small workspace and of misaligned or short buffers."""
+the h = H^I invariant (MISA page, Eq. 9 with every head routed is Eq. 1), the timed
+scorer entry the benchmark's roofline uses, and the host-side rejection of a too-small
+workspace and of misaligned or short buffers."""
 
 import ctypes
 
@@ -205,3 +206,24 @@ def test_workspace_too_small_and_bad_buffers_rejected(M):
                                        wl.h, wl.topk, P(host_idx), None, None, st) == 1
     torch.cuda.synchronize()
     assert bool((idx == -7).all())
+
+
+@pytest.mark.parametrize("T", [1, 64], ids=["decode_form", "block_form"])
+def test_timed_scorer_matches_score_rows(M, T):
+    # the timed entry runs the same scorer as misa_score_rows: identical scores (the
+    # same kernel on the same inputs), and a positive kernel time
+    wl = _wl(T=T, L=4096, pos_mode="tail" if T == 1 else "causal")
+    if T > 1:
+        wl = wl.replace(L=T)
+    x = make_inputs(wl, seed=5)
+    q, w, k, pos = gpu_path.to_device(x)
+    kp = M.misa_pool_keys(k, wl.B)
+    heads = M.misa_route_heads(q, w, k, kp, pos, wl.B, wl.h)
+    ref = M.misa_score_rows(q, w, k, heads, pos)
+    out = torch.full_like(ref, float("nan"))
+    ms = M.misa_testing_score_rows_timed(q, w, k, heads, pos, scores=out)
+    M.misa_check_device_status(q.device)
+    assert ms > 0.0
+    P = pos.long() + 1
+    valid = torch.arange(ref.shape[-1], device=ref.device)[None, None, :] < P[..., None]
+    assert torch.equal(out[valid], ref[valid])

@@ -15,10 +15,9 @@
 // MMAs reproduce the fp32 products to about 2^-16 relative.  Accumulators live in TMEM
 // (N = the item's largest full-block count within its chunk, rounded up to 16).
 //
-// Epilogue: two groups of 4 warps (one per TMEM lane quarter); group g serves the tiles
-// t0 + g, t0 + g + 2, ... with its own pair of 128-column accumulators, so the two groups'
-// per-tile latency chains overlap and the MMAs of a group's next item run while it reads the
-// current one.  Each warp owns 32 (query, head) rows of its tile: the partial-block dot
+// Epilogue: four groups of 4 warps (one per TMEM lane quarter); group g serves the tiles
+// t0 + g, t0 + g + 4, ... with its own 128-column accumulator, so four tiles' per-tile
+// latency chains overlap (and the MMAs of one group's item run while the others read theirs).  Each warp owns 32 (query, head) rows of its tile: the partial-block dot
 // product reads the query row from the tile's A stage (released by the epilogue, not by the
 // MMA) and the tile's partial pooled keys from a shared-memory copy loaded with the A tile;
 // then the row's ReLU sum over its causal block count, E (written when asked for), and a
@@ -46,9 +45,9 @@ constexpr int kBBytes = kMaxBlocks * kHeadDim * 2;  // 64 KB per part (hi or lo)
 constexpr int kBHalf = kBBytes / 2;
 constexpr int kMaxQT = 16;                          // queries per tile (H >= 8)
 constexpr int kKpBytes = kMaxQT * kHeadDim * 4;     // partial pooled keys of a tile (fp32)
-constexpr int kGroups = 2;                          // epilogue groups
-constexpr int kStages = kGroups;                    // stage s holds the tiles group s serves
-constexpr int kAccPerGroup = 2;
+constexpr int kGroups = 4;                          // epilogue groups
+constexpr int kStages = 2;
+constexpr int kAccPerGroup = 1;
 constexpr int kAcc = kGroups * kAccPerGroup;
 constexpr int kCols = kAcc * kItemBlocks;           // 512
 constexpr int kGroupThreads = 128;
@@ -62,12 +61,16 @@ constexpr int kBBase = kStages * kATileBytes;         // hi then lo
 constexpr int kKpBase = kBBase + 2 * kBBytes;
 constexpr int kEsBase = kKpBase + kStages * kKpBytes;  // E of a tile's rows: [group][2][kRows]
 constexpr int kBarBase = kEsBase + kGroups * 2 * kRows * 4;
-// full[S], empty[S], bfull, bempty, accfull[A], accempty[A], drain
-constexpr int kNumBars = 2 * kStages + 2 + 2 * kAcc + 1;
+// full[G] (per epilogue group: a group's tiles complete its phases one by one, so its
+// parity waits never alias a stage's later tile), empty[S], bfull, bempty, accfull[A],
+// accempty[A], drain
+constexpr int kNumBars = kGroups + kStages + 2 + 2 * kAcc + 1;
 constexpr int kMiscBase = kBarBase + kNumBars * 8;
-constexpr int kSmemBytes = kMiscBase + 16 + 1024;
+constexpr int kMetaTiles = 1024;                       // tiles whose block counts are staged
+constexpr int kMetaBase = kMiscBase + 16;              // per-tile full-block counts [kMetaTiles]
+constexpr int kSmemBytes = kMetaBase + kMetaTiles * 4 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-static_assert(kStages == kGroups && kGroups == 2 && kMaxBlocks == 2 * kItemBlocks, "tile-to-group map");
+static_assert(kGroups % kStages == 0 && kMaxBlocks == 2 * kItemBlocks, "tile-to-group map");
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
   volatile int never = 0;
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kBarBase);
-  uint64_t* empty = full + kStages;
+  uint64_t* empty = full + kGroups;
   uint64_t* bfull = empty + kStages;
   uint64_t* bempty = bfull + 1;
   uint64_t* accfull = bempty + 1;
@@ -153,10 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kMiscBase);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kMiscBase + 4);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+    for (int g2 = 0; g2 < kGroups; ++g2) mbar_init(&full[g2], 1);
+    for (int s = 0; s < kStages; ++s)
       mbar_init(&empty[s], 1 + 4);   // the MMAs' commit and the serving group's warps
-    }
     mbar_init(bfull, 1);
     mbar_init(bempty, 1);
     for (int a = 0; a < kAcc; ++a) {
@@ -168,6 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kCols);
+  // Every tile's largest full-block count, loaded once by all threads (its queries' prefix
+  // lengths) so that the producer and the MMA issuer do not wait on them tile by tile.
+  int* meta = reinterpret_cast<int*>(base + kMetaBase);
+  const bool staged = t1 - t0 <= kMetaTiles;
+  if (staged)
+    for (int j = tid; j < t1 - t0; j += kThreads) meta[j] = tile_blocks(pos, g, t0 + j);
+  auto blocks_of = [&](int i) { return staged ? meta[i - t0] : tile_blocks(pos, g, i); };
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -188,12 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
           break;
         uint8_t* ab = base + kStageBase + s * kATileBytes;
         const int64_t qrow0 = (int64_t)n * g.T + (int64_t)(i % g.tiles_per_seq) * g.QT;
-        mbar_arrive_expect_tx(&full[s], kATileBytes + kp_bytes);
-        tma_load_2d(ab, &tm_q, &full[s], 0, i * kRows);
-        tma_load_2d(ab + kAHalf, &tm_q, &full[s], 64, i * kRows);
-        bulk_load(base + kKpBase + s * kKpBytes, kpart + qrow0 * kHeadDim, kp_bytes, &full[s]);
+        uint64_t* fb = &full[issued % kGroups];   // the serving group's barrier
+        mbar_arrive_expect_tx(fb, kATileBytes + kp_bytes);
+        tma_load_2d(ab, &tm_q, fb, 0, i * kRows);
+        tma_load_2d(ab + kAHalf, &tm_q, fb, 64, i * kRows);
+        bulk_load(base + kKpBase + s * kKpBytes, kpart + qrow0 * kHeadDim, kp_bytes, fb);
         ++issued;
-        const int nc = tile_items(tile_blocks(pos, g, i));
+        const int nc = tile_items(blocks_of(i));
         for (int k = 0; k < nc; ++k) {
           const int c = item_chunk(i, k, nc);
           const int64_t key = (int64_t)n * 65536 + c;
@@ -218,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     __syncthreads();   // (A)
     if (lane == 0) {
       for (int i = max(0, issued - kStages); i < issued; ++i)
-        drain_wait(&full[i % kStages], (i / kStages) & 1, status);
+        drain_wait(&full[i % kGroups], (i / kGroups) & 1, status);
       if (bissued) drain_wait(bfull, (bissued - 1) & 1, status);
     }
     __syncthreads();   // (B)
@@ -227,14 +237,14 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     if (lane == 0) {
       const uint32_t smem0 = smem_u32(base);
       int it = 0, bseen = 0;
-      int uses0 = 0, uses1 = 0;   // items issued for each group's accumulator pair
+      int uses[kGroups] = {};   // items issued for each group's accumulators
       int64_t cur_key = -1;
       bool ok = true;
       for (int i = t0; i < t1 && ok; ++i) {
         const int n = i / g.tiles_per_seq;
         const int s = it % kStages, grp = it % kGroups;
-        if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, status, kWaitCycles)) break;
-        const int mf = tile_blocks(pos, g, i);
+        if (!mbar_wait(&full[grp], (it / kGroups) & 1, abort_flag, status, kWaitCycles)) break;
+        const int mf = blocks_of(i);
         const int nc = tile_items(mf);
         for (int k = 0; k < nc && ok; ++k) {
           const int c = item_chunk(i, k, nc);
@@ -250,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
           }
           for (int sub = 0; sub < kMaxBlocks / kItemBlocks && ok; ++sub) {
             if (!item_present(c, sub, mf)) continue;
-            const int u = grp ? uses1++ : uses0++;
+            const int u = uses[grp]++;
             const int acc = grp * kAccPerGroup + (u % kAccPerGroup);
             if (!mbar_wait(&accempty[acc], ((u / kAccPerGroup) & 1) ^ 1, abort_flag, status,
                            kWaitCycles)) {
@@ -294,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
     tc_fence_after();
     tmem_dealloc(tmem_base, kCols);
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9)
-    const int grp = (warp - 2) >> 2;     // group: tiles t0 + grp, t0 + grp + 2, ...
+    // ------------------------------------------------------------ epilogue (warps 2 ..)
+    const int grp = (warp - 2) >> 2;     // group: tiles t0 + grp, t0 + grp + kGroups, ...
     const int quarter = warp & 3;        // TMEM lanes this warp may read
     const int r = quarter * 32 + lane;   // row of the tile
     const int qq = r / g.H, j = r % g.H;
@@ -338,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
       // the partial last block: q . kpart over 128 dimensions, reading the query row from
       // the tile's A stage and the partial keys copied with it, then releasing the stage
       float dot = 0.f;
-      if (ok && !warp_wait(&full[s], (it / kStages) & 1, abort_flag, status)) ok = false;
+      if (ok && !warp_wait(&full[grp], (it / kGroups) & 1, abort_flag, status)) ok = false;
       if (ok && M > mfull) {
         float d4[4] = {0.f, 0.f, 0.f, 0.f};   // four chains, so the FMAs overlap
 #pragma unroll

@@ -46,6 +46,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (instead of returning at once) until
+// the phase completes or about `suspend_ns` nanoseconds have passed, so that a CTA whose
+// threads all wait does not spend issue slots polling.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity,
+                                                      uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Longest single suspension inside mbar_wait: the abort flag and the cycle limit are
+// checked between suspensions.
+constexpr uint32_t kSuspendNs = 10000;
+
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_cycles` SM clock cycles (or when another role already gave up), records
 // MISA_ERR_DEVICE_TIMEOUT in the global status word and returns false.
@@ -54,7 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > limit_cycles) {
       *abort_flag = 1;

@@ -676,6 +676,7 @@ __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
 constexpr int kRowCap = 16384;
 constexpr int kLongRowCap = 40960;
 constexpr long long kRowWaitCycles = 4000000000LL;
+constexpr uint32_t kRowSuspendNs = 20000;   // longest single suspension in the copy wait
 
 template <int NT, int CAP, int ROWCAP>
 struct RowCfg {
@@ -794,9 +795,9 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     C = s_total;
   }
   bool landed = true;
-  if (nbulk > 0) {   // bounded wait for the copy
+  if (nbulk > 0) {   // bounded wait for the copy (threads sleep in the wait, not spin)
     long long t0 = clock64();
-    while (!sm100::mbar_try_wait(&lbar, 0)) {
+    while (!sm100::mbar_try_wait_suspend(&lbar, 0, kRowSuspendNs)) {
       if (clock64() - t0 > kRowWaitCycles) {
         landed = false;
         break;
@@ -806,7 +807,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
       if (t == 0) set_status(status, MISA_ERR_DEVICE_TIMEOUT);
       t0 = clock64();
       landed = true;
-      while (!sm100::mbar_try_wait(&lbar, 0)) {
+      while (!sm100::mbar_try_wait_suspend(&lbar, 0, kRowSuspendNs)) {
         if (clock64() - t0 > kRowWaitCycles) {
           landed = false;
           break;

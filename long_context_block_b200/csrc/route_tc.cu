@@ -420,15 +420,17 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(
       // that rank when the rank is below h
       if (ok && valid) {   // H is a multiple of 8: four energies per load
         const float4* eq = reinterpret_cast<const float4*>(Es + qq * g.H);
-        int rank = 0;
+        int rk0 = 0, rk1 = 0;   // two counts, loads four steps ahead
+#pragma unroll 4
         for (int j4 = 0; j4 < g.H / 4; ++j4) {
           const float4 o = eq[j4];
           const int jb = 4 * j4;
-          rank += (o.x > ev || (o.x == ev && jb < j)) ? 1 : 0;
-          rank += (o.y > ev || (o.y == ev && jb + 1 < j)) ? 1 : 0;
-          rank += (o.z > ev || (o.z == ev && jb + 2 < j)) ? 1 : 0;
-          rank += (o.w > ev || (o.w == ev && jb + 3 < j)) ? 1 : 0;
+          rk0 += (o.x > ev || (o.x == ev && jb < j)) ? 1 : 0;
+          rk1 += (o.y > ev || (o.y == ev && jb + 1 < j)) ? 1 : 0;
+          rk0 += (o.z > ev || (o.z == ev && jb + 2 < j)) ? 1 : 0;
+          rk1 += (o.w > ev || (o.w == ev && jb + 3 < j)) ? 1 : 0;
         }
+        const int rank = rk0 + rk1;
         if (rank < h) heads[qrow * h + rank] = j;
       }
     }

@@ -952,17 +952,16 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
     // one-pass compaction: warp w takes the row's key steps w, w + kWarps, ... (an even
     // sample of the row) and appends its candidates to its own region, then to the pool
     // and the spill area; every candidate is counted in its sub-bucket, stored or not
-    auto put = [&](uint32_t r, uint32_t key, int ee) {
+    // candidate of rank r in this warp's region: store it there, or at overflow slot o
+    // (pool, then spill area) when r >= kReg
+    auto put = [&](uint32_t r, uint32_t o, uint32_t key, int ee) {
       atomicAdd(&sub[bpad(bucket_of(key))], 1u);
-      if (r < kReg) {
+      if (r < kReg)
         cand[warp * kReg + r] = compose(key, ee);
-      } else {
-        const uint32_t p = atomicAdd(&s_spill, 1u);
-        if (p < kPool)
-          pool[p] = compose(key, ee);
-        else if (p - kPool < spill_cap)
-          spill[p - kPool] = compose(key, ee);
-      }
+      else if (o < kPool)
+        pool[o] = compose(key, ee);
+      else if (o - kPool < spill_cap)
+        spill[o - kPool] = compose(key, ee);
     };
     uint32_t wc = 0;
     if (hb == 0) {   // 128-key steps: lane l takes keys e .. e + 3
@@ -985,11 +984,28 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
         const uint32_t b1 = __ballot_sync(0xffffffffu, c & 2u);
         const uint32_t b2 = __ballot_sync(0xffffffffu, c & 4u);
         uint32_t r = wc + __popc(b0 & below) + 2u * __popc(b1 & below) + 4u * __popc(b2 & below);
-        if (t0) put(r++, v.x, e);
-        if (t1) put(r++, v.y, e + 1);
-        if (t2) put(r++, v.z, e + 2);
-        if (t3) put(r++, v.w, e + 3);
-        wc += __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
+        const uint32_t step = __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
+        // ranks at or past kReg overflow: one shared-counter add per warp step, each lane's
+        // overflowing pairs in rank order after the lower lanes' ones
+        uint32_t o = 0u;
+        if (wc + step > kReg) {
+          const uint32_t first = max(r, kReg), last = max(r + c, kReg);
+          const uint32_t mine = last - first;   // 0 .. 4
+          const uint32_t o0 = __ballot_sync(0xffffffffu, mine & 1u);
+          const uint32_t o1 = __ballot_sync(0xffffffffu, mine & 2u);
+          const uint32_t o2 = __ballot_sync(0xffffffffu, mine & 4u);
+          const uint32_t tot = __popc(o0) + 2u * __popc(o1) + 4u * __popc(o2);
+          uint32_t base = 0u;
+          if (lane == 0) base = atomicAdd(&s_spill, tot);
+          base = __shfl_sync(0xffffffffu, base, 0);
+          o = base + __popc(o0 & below) + 2u * __popc(o1 & below) + 4u * __popc(o2 & below);
+          o -= first - r;   // so that the pair of rank q >= kReg gets o + (q - r)
+        }
+        if (t0) { put(r, o, v.x, e); ++r; ++o; }
+        if (t1) { put(r, o, v.y, e + 1); ++r; ++o; }
+        if (t2) { put(r, o, v.z, e + 2); ++r; ++o; }
+        if (t3) { put(r, o, v.w, e + 3); ++r; ++o; }
+        wc += step;
       }
     } else {   // 32-key steps
 #pragma unroll 4
@@ -998,7 +1014,10 @@ __global__ void __launch_bounds__(NT, MINB) topk_row_kernel(
         const uint32_t key = e < n ? keys[e] : 0u;
         const bool take = e < n && key >= kcut;
         const uint32_t m = __ballot_sync(0xffffffffu, take);
-        if (take) put(wc + __popc(m & below), key, e);
+        const uint32_t r = wc + __popc(m & below);
+        uint32_t o = 0u;
+        if (take && r >= kReg) o = atomicAdd(&s_spill, 1u);
+        if (take) put(r, o, key, e);
         wc += __popc(m);
       }
     }

@@ -9,13 +9,13 @@
 // key is the mean of its valid keys only, computed here from the raw keys.
 //
 // For queries that do not share a sequence with many others (decode): every query row is
-// a thread-block cluster of up to 8 CTAs.  Each CTA stages the query's head vectors once
-// and walks its share of the prefix's chunks of kRouteChunk blocks: the chunk's pooled
-// keys go to shared memory split into bf16 hi + lo parts, q_j . kp_b runs on the tensor
-// cores (mma.sync, fp32 accumulators), and the CTA adds sum_b ReLU(q_j . kp_b) into its
-// per-head sums.  CTA 0 of the cluster then sums the members' partial sums through
-// distributed shared memory, applies |w_j| / M_t (common to all blocks, so applied once),
-// writes E and selects the top-h heads by repeated warp arg-max.
+// a thread-block cluster of up to 16 CTAs (8 where a device cannot hold 16).  Each CTA
+// stages the query's head vectors once and walks its share of the prefix's chunks of
+// kRouteChunk blocks: the chunk's pooled keys go to shared memory split into bf16 hi + lo
+// parts, q_j . kp_b runs on the tensor cores (mma.sync, fp32 accumulators), and the CTA
+// adds sum_b ReLU(q_j . kp_b) into its per-head sums.  CTA 0 of the cluster then sums the
+// members' partial sums through distributed shared memory, applies |w_j| / M_t (common to
+// all blocks, so applied once), writes E and selects the top-h heads.
 //
 // The same products, in the block-score mode, reduce the affinities along the other axis
 // for the HISA-style token-axis filter (MISA page, "Key distinction from HISA"):
@@ -33,7 +33,8 @@ namespace {
 namespace cg = cooperative_groups;
 
 constexpr int kCh = kRouteChunk;
-constexpr int kMaxCluster = 8;   // CTAs per query row (portable cluster size)
+constexpr int kMaxCluster = 16;  // CTAs per query row (16: non-portable, where it fits)
+constexpr int kPortableCluster = 8;
 
 // (value desc, index asc) ordering for the warp arg-max.
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
@@ -356,11 +357,33 @@ cudaError_t launch_route_mt(const uint16_t* q, const float* w, const uint16_t* k
                             cudaStream_t st) {
   const int Mpool = (int)((L + B - 1) / B);
   const int nchunk = (Mpool + kCh - 1) / kCh;
-  const int CS = nchunk < kMaxCluster ? nchunk : kMaxCluster;
+  int CS = nchunk < kMaxCluster ? nchunk : kMaxCluster;
   const size_t smem = route_smem_bytes<MT>();
   cudaError_t err = cudaFuncSetAttribute(route_kernel<MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
+  if (CS > kPortableCluster) {
+    // clusters of more than 8 CTAs only where the device can hold one
+    int nclusters = 0;
+    cudaLaunchConfig_t q16 = {};
+    q16.gridDim = dim3((unsigned)CS, 1, 1);
+    q16.blockDim = dim3(kRouteThreads, 1, 1);
+    q16.dynamicSmemBytes = smem;
+    cudaLaunchAttribute a16[1];
+    a16[0].id = cudaLaunchAttributeClusterDimension;
+    a16[0].val.clusterDim.x = (unsigned)CS;
+    a16[0].val.clusterDim.y = 1;
+    a16[0].val.clusterDim.z = 1;
+    q16.attrs = a16;
+    q16.numAttrs = 1;
+    if (cudaFuncSetAttribute(route_kernel<MT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&nclusters, route_kernel<MT>, &q16) != cudaSuccess ||
+        nclusters < 1) {
+      cudaGetLastError();
+      CS = kPortableCluster;
+    }
+  }
   for (int64_t row0 = 0; row0 < rows; row0 += 65535) {
     const int64_t nr = rows - row0 < 65535 ? rows - row0 : 65535;
     cudaLaunchConfig_t cfg = {};

@@ -357,7 +357,12 @@ cudaError_t launch_route_mt(const uint16_t* q, const float* w, const uint16_t* k
                             cudaStream_t st) {
   const int Mpool = (int)((L + B - 1) / B);
   const int nchunk = (Mpool + kCh - 1) / kCh;
-  int CS = nchunk < kMaxCluster ? nchunk : kMaxCluster;
+  // 16 CTAs per row only for few rows (else the extra members cost more than they share)
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int cap = (int64_t)rows * kMaxCluster <= 4LL * sms ? kMaxCluster : kPortableCluster;
+  int CS = nchunk < cap ? nchunk : cap;
   const size_t smem = route_smem_bytes<MT>();
   cudaError_t err = cudaFuncSetAttribute(route_kernel<MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -8,7 +8,8 @@
 // topk_row_kernel (rows up to 16384 scores, or 40960 with the scorer's histogram): one CTA
 // per row stages the row in shared memory with one bulk copy, finds the cutoff bin of a
 // 12-bit key histogram (refined by the next 12 bits when the bin is crowded), compacts the
-// candidates and sorts them with a histogram-adaptive counting sort (groupsort.cuh).
+// candidates while counting them into sub-buckets of the bins above the cutoff, and places
+// every pair by a scan, a scatter and a rank inside its bucket.
 //
 // topk_scatter_kernel + topk_group_kernel (longer decode rows with the scorer's histogram):
 // many CTAs per row append the candidates to groups of output positions, one CTA per group
@@ -667,9 +668,11 @@ __global__ void __launch_bounds__(kThreads) topk_hist_overflow_kernel(
 // into shared memory with one bulk asynchronous copy (plain loads for the at most three
 // scores on either side of its 16-byte-aligned interior), turns the scores into keys in
 // place, finds the cutoff bin with a histogram of the top kScoreHistBits key bits (or
-// takes the one the scorer built), compacts the candidates (bins at or above it) and
-// sorts them with the counting sort.  A crowded cutoff (more than CAP candidates) takes
-// an exact radix select over the resident keys instead.  Shapes: 256 threads, 3072
+// takes the one the scorer built), compacts the candidates (bins at or above it) counting
+// them into sub-buckets, and writes each at the output position that a scan of the bucket
+// counts, a scatter into bucket order and a rank inside the bucket give it.  A crowded
+// cutoff (more than CAP candidates) takes an exact radix select over the resident keys
+// and the adaptive counting sort (groupsort.cuh) instead.  Shapes: 512 threads, 3072
 // candidates, 16K rows (two CTAs per SM: many rows, k <= 3072); 512 or 1024 threads, 8192
 // candidates, 16K rows (one CTA per SM; 1024 threads when rows are too few to fill the
 // SMs); 1024 threads, 3072 candidates, 40K rows (long decode rows).

@@ -194,12 +194,14 @@ def test_tied_long_rows_exact_fallback(M):
         assert torch.equal(idx.cpu(), ref) and torch.equal(didx.cpu(), ref), kk
 
 
-def test_dagger_candidates_any_order_with_repeats(M):
+@pytest.mark.parametrize("L", [2000, 40000], ids=["one_cta_per_row", "cluster_split_rows"])
+def test_dagger_candidates_any_order_with_repeats(M, L):
     """Eq. (12) re-scores the set Omega_t: candidates given shuffled, with repeated ids
-    and empty slots, re-rank exactly like the oracle on the distinct ids."""
+    and empty slots, re-rank exactly like the oracle on the distinct ids (at L = 40000 the
+    six rows' candidate ordering splits each prefix over a cluster of CTAs)."""
     import oracle.misa_oracle as orc
     from tests import tolerance as tl
-    wl = _wl(nseq=2, T=3, L=2000, topk=64, kprime=400)
+    wl = _wl(nseq=2, T=3, L=L, topk=64, kprime=400)
     x = make_inputs(wl, seed=21)
     rng = np.random.default_rng(8)
     cand = np.full((wl.nseq, wl.T, wl.kprime), -1, dtype=np.int32)

@@ -53,3 +53,20 @@ def test_forms_and_launch_counts():
     assert bench.misa_step_launches(WORKLOADS["dsv32_mtp_32k"]) == 6
     # prefill: three tensor-core router kernels (hi/lo split, partial blocks, GEMM + top-h)
     assert bench.misa_step_launches(WORKLOADS["dsv32_prefill_16k"]) == 7
+
+
+def test_roofline_object_from_a_kernel_time():
+    # 32K decode: HBM-bound; achieved = algorithmic bytes / kernel time, frac against the
+    # measured copy peak; the traffic figure passes through unchanged
+    peaks = {"hbm": 6557.4, "bf16": 1629.0, "source": "measured"}
+    wl = WORKLOADS["dsv32_decode_32k"]
+    r = bench._roofline(wl, 0.0544, peaks, 274656768)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 274656768
+    assert abs(r["achieved"] - bench.algorithmic_bytes_score(wl) / 0.0544e-3 / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6557.4) < 1e-12 and 0.7 < r["frac"] < 0.8
+    # 16K prefill: tensor-bound against the bf16 burst peak
+    wl = WORKLOADS["dsv32_prefill_16k"]
+    r = bench._roofline(wl, 0.3057, peaks, None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["traffic"] is None
+    assert abs(r["achieved"] - bench.algorithmic_flops_score(wl) / 0.3057e-3 / 1e12) < 1e-6
+    assert 0.5 < r["frac"] < 0.6
